@@ -1,0 +1,416 @@
+#!/usr/bin/env python
+"""Benchmark of the routed MoE expert forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pass of the whole hot path on one batch of synthetic input:
+moe_route (router top-k) followed by moe_forward (permute, gate/up with
+SwiGLU, down, combine) of one layer. The default workload is the
+decode-shaped layer (T=16, H=2048, I=1408, E=60, k=4, bf16); --workload picks
+another (tiny, decode, prefill, fp8, skewed).
+
+Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events
+on the launching stream, with a 256 MiB buffer written between steps (outside
+the events) so that no step finds the previous step's data in L2. Inputs are
+resident in HBM when a step starts. Multi-GPU (torchrun, one process per GPU)
+runs independent replicas: the layer has no data-path exchange; the elapsed
+time is the max over ranks and the value counts the tokens of all ranks.
+
+The JSON line also carries: the stage breakdown (events recorded by
+moe_forward_timed), the roofline of the dominant kernel (algorithmic bytes or
+FLOPs per launch over its measured duration, against MEASURED_PEAKS.json),
+the end-to-end number through the public API with host buffers (H2D of x and
+logits, D2H of the output inside the timed region), the CPU oracle timed on a
+bounded sample (rank 0, N=1), the number of our kernel launches in the timed
+region, and the SM clocks sampled during it.
+
+--impl reference times the CPU oracle (test infrastructure, unmodified) on the
+same workload, a bounded sample of tokens per step, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from mixture_experts_routed_moe_b200 import inputs as G  # noqa: E402
+
+METRIC = "MoE layer tokens/sec and TFLOP/s (% of BF16/FP8 peak or HBM BW) on 1 B200"
+DEFAULT_WORKLOAD = "decode"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FLUSH_BYTES = 256 << 20
+
+# DRAM traffic per launch of the dominant kernel, from one ncu capture, keyed by
+# (workload, kernel) together with the hash of the kernel's source file at the
+# time of the capture; a changed source makes the figure stale (reported null).
+NCU_TRAFFIC = {}
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def src_hash(name):
+    path = os.path.join(ROOT, "mixture_experts_routed_moe_b200", "csrc", name)
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.file = None
+
+    def start(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.file, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.file.flush()
+        self.file.seek(0)
+        rows = [r.split(",") for r in self.file.read().strip().splitlines() if r.strip()]
+        os.unlink(self.file.name)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+                for n, v in zip(names, r[5:9]):
+                    if v.strip().lower() == "active":
+                        reasons.add(n)
+            except (ValueError, IndexError):
+                continue
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_init(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(v, world):
+    if world == 1:
+        return v
+    import torch.distributed as dist
+
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (the baseline and the reference arm)
+# ---------------------------------------------------------------------------
+
+class _HostExperts:
+    """Host copies of the experts a sample touches (made outside the timing)."""
+
+    def __init__(self, wl, seed, experts, name, codes=False):
+        dev = "cuda" if torch.cuda.is_available() else "cpu"
+        self.shape = {"w_gate_up": (wl.E, 2 * wl.I, wl.H), "w_down": (wl.E, wl.H, wl.I),
+                      "sw_gate_up": (wl.E, 2 * wl.I // 128, wl.H // 128),
+                      "sw_down": (wl.E, wl.H // 128, wl.I // 128)}[name]
+        self.d = {}
+        for e in experts:
+            t = G.make_expert_weights(wl, seed, int(e), device=dev)[name].cpu()
+            self.d[int(e)] = t.view(torch.uint8).numpy() if codes else t.float().numpy()
+
+    def __getitem__(self, e):
+        return self.d[int(e)]
+
+
+def oracle_sample_rate(wl, seed, n_tokens, steps=1, warmup=0):
+    """Times the oracle's route + eager forward on the first n_tokens tokens.
+    Returns (tokens/s, seconds per step, BLAS threads)."""
+    from oracle import moe_oracle as O
+
+    x, logits = G.make_activations(wl, seed)
+    toks = np.arange(min(n_tokens, wl.T))
+    L = logits.numpy()[toks]
+    xs = x.float().numpy()[toks]
+    idx0, _, _ = O.route(L, wl.k)
+    experts = np.unique(idx0)
+    fp8 = wl.wdtype == "e4m3"
+    V = {n: _HostExperts(wl, seed, experts, n, codes=fp8) for n in
+         (("w_gate_up", "w_down", "sw_gate_up", "sw_down") if fp8 else ("w_gate_up", "w_down"))}
+    times = []
+    for i in range(warmup + steps):
+        t0 = time.perf_counter()
+        idx, w, _ = O.route(L, wl.k)
+        if fp8:
+            O.moe_forward_fp8(xs, idx, w, V["w_gate_up"], V["sw_gate_up"], V["w_down"], V["sw_down"])
+        else:
+            O.moe_forward(xs, idx, w, V["w_gate_up"], V["w_down"])
+        if i >= warmup:
+            times.append(time.perf_counter() - t0)
+    try:
+        from threadpoolctl import threadpool_info
+
+        threads = max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
+    except Exception:
+        threads = os.cpu_count() or 1
+    per_step = sum(times) / len(times)
+    return len(toks) / per_step, per_step, threads, times
+
+
+def oracle_sample_tokens(wl):
+    return min(wl.T, 16)
+
+
+def run_reference(args, world, rank):
+    wl = G.WORKLOADS[args.workload]
+    if rank != 0:
+        return
+    n = oracle_sample_tokens(wl)
+    rate, per_step, threads, times = oracle_sample_rate(wl, G.default_seed(wl), n, steps=args.steps,
+                                                        warmup=args.warmup)
+    sample = f"first {n} of {wl.T} tokens per step (route + eager expert loop + combine, float64 NumPy)"
+    line = {
+        "metric": METRIC, "impl": "reference", "value": rate, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(wl, "oracle"),
+        "cpu_baseline": {"value": rate, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": rate, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def workload_config(wl, path):
+    return {"workload": wl.name, "T": wl.T, "H": wl.H, "I": wl.I, "E": wl.E, "k": wl.k, "wdtype": wl.wdtype,
+            "path": path, "l2": "flushed between steps (256 MiB write)", "parallelism": "replicas"}
+
+
+def stage_roofline(wl, path, stage_ms, n_touched, peaks, peak_src):
+    """Roofline of the slowest stage (its one kernel), algorithmic work per launch."""
+    A, H, I = wl.A, wl.H, wl.I
+    welem = 1 if wl.wdtype == "e4m3" else 2
+    names = {1: "gate_up", 2: "down"}
+    s = max((1, 2), key=lambda i: stage_ms[i])
+    dur_s = stage_ms[s] / 1e3
+    if path == "decode":
+        if s == 1:
+            byts = n_touched * 2 * I * H * welem + wl.T * H * 2 + A * I * 2
+            kern, src = "decode_gate_up_kernel", "decode.cu"
+        else:
+            byts = n_touched * H * I * welem + A * I * 2 + A * H * 2
+            kern, src = "decode_down_kernel", "decode.cu"
+        ach = byts / dur_s / 1e9
+        peak = peaks["hbm_gbs"]
+        out = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
+               "kernel": kern, "stage": names[s], "algorithmic_bytes": byts}
+    else:
+        flops = (4 if s == 1 else 2) * A * H * I
+        ach = flops / dur_s / 1e12
+        if wl.wdtype == "e4m3":
+            peak, how = 2.0 * peaks["bf16_tflops"], "2x measured bf16 (nominal fp8:bf16 ratio)"
+            kern, src = ("gemm_e4m3_gate_up" if s == 1 else "gemm_e4m3_down"), "gemm_e4m3.cu"
+        else:
+            peak, how = peaks["bf16_tflops"], "measured bf16 burst"
+            kern, src = ("grouped_gemm_bf16_kernel<256,true>" if s == 1 else "grouped_gemm_bf16_kernel<256,false>"), \
+                "gemm_bf16.cu"
+        out = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
+               "kernel": kern, "stage": names[s], "algorithmic_flops": flops, "peak_source": how}
+    rec = NCU_TRAFFIC.get((wl.name, kern))
+    out["traffic"] = rec["bytes"] if rec and rec["src"] == src_hash(src) else None
+    out["peak_from"] = peak_src
+    return out
+
+
+def run_ours(args, world, rank, local):
+    import mixture_experts_routed_moe_b200 as moe
+
+    wl = G.WORKLOADS[args.workload]
+    seed = G.default_seed(wl)
+    dev = torch.device("cuda", local if world > 1 else 0)
+    x, logits = G.make_activations(wl, seed)
+    W = G.make_weights(wl, seed, device=dev)
+    xd, ld = x.to(dev), logits.to(dev)
+    layer = moe.MoELayer(W["w_gate_up"], W["w_down"], wl.k, W.get("sw_gate_up"), W.get("sw_down"))
+    out = torch.empty((wl.T, wl.H), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    shape = moe.make_shape(wl.T, wl.H, wl.I, wl.E, wl.k, wl.wdtype, "auto")
+    lay = moe.workspace_layout(shape)
+    path = moe.PATH_NAMES[lay.path]
+    stream = torch.cuda.current_stream()
+
+    def new_events(n):
+        return [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        layer(xd, ld, out=out)
+    torch.cuda.synchronize()
+    ws = layer._workspace(wl.T, dev)
+    if moe.read_device_status(ws) != 0:
+        raise RuntimeError("device status reports an error after warm-up")
+    n_touched = int(ws[lay.hdr:lay.hdr + 12].view(torch.int32)[1].item())
+
+    K = args.steps
+    ev_s, ev_e = new_events(K), new_events(K)
+    st_ev = [new_events(5) for _ in range(K)]
+    clocks = ClockSampler(dev.index)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    for i in range(K):
+        flush.zero_()
+        ev_s[i].record(stream)
+        layer(xd, ld, out=out, events=st_ev[i])
+        ev_e[i].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    step_ms = [ev_s[i].elapsed_time(ev_e[i]) for i in range(K)]
+    total_ms = max_over_ranks(sum(step_ms), world)
+    stage_ms = {j: sum(st_ev[i][j - 1].elapsed_time(st_ev[i][j]) for i in range(K)) / K for j in range(1, 5)}
+    route_ms = sum(ev_s[i].elapsed_time(st_ev[i][0]) for i in range(K)) / K
+
+    # end to end through the public API with host buffers
+    xh = x.pin_memory()
+    lh = logits.pin_memory()
+    oh = torch.empty((wl.T, wl.H), dtype=torch.bfloat16).pin_memory()
+    xd2, ld2 = torch.empty_like(xd), torch.empty_like(ld)
+    e2e_s, e2e_e = new_events(K), new_events(K)
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(K):
+        flush.zero_()
+        e2e_s[i].record(stream)
+        xd2.copy_(xh, non_blocking=True)
+        ld2.copy_(lh, non_blocking=True)
+        layer(xd2, ld2, out=out)
+        oh.copy_(out, non_blocking=True)
+        e2e_e[i].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(sum(e2e_s[i].elapsed_time(e2e_e[i]) for i in range(K)), world)
+
+    peaks, peak_src = load_peaks()
+    per_step_launches = 1 + (1 if wl.T <= 256 else 3) + 2 + 1  # route, permute, gate/up, down, combine
+    if wl.wdtype == "e4m3":
+        per_step_launches += 1  # activation quantisation
+    tokens = wl.T * K * world
+    value = tokens / (total_ms / 1e3)
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": wl.wdtype, "data": "synthetic (seeded N(0,1) activations and logits, N(0,0.02) weights)",
+        "config": workload_config(wl, path),
+        "tflops": wl.flops() * K * world / (total_ms / 1e3) / 1e12,
+        "stages_ms": {"route": route_ms, "permute": stage_ms[1], "gate_up": stage_ms[2], "down": stage_ms[3],
+                      "combine": stage_ms[4]},
+        "touched_experts": n_touched,
+        "roofline": roof,
+        "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": x.numel() * 2 + logits.numel() * 4, "d2h_bytes_per_step": wl.T * wl.H * 2},
+        "gpu_launches": per_step_launches * K,
+        "clocks": clk,
+    }
+    # stage indices above: events[0..4] = before permute, after permute, after gate/up, after down, after combine
+    line["roofline"] = stage_roofline(wl, path, {1: stage_ms[2], 2: stage_ms[3]}, n_touched, peaks, peak_src)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n = oracle_sample_tokens(wl)
+        rate, per_step, threads, _ = oracle_sample_rate(wl, seed, n, steps=1, warmup=0)
+        line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                                "sample": f"first {n} of {wl.T} tokens, one pass ({per_step:.2f} s)"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=list(G.WORKLOADS), default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        log("note: fewer than 3 warm-up steps")
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, world, rank)
+        return
+    world, rank, local = dist_init(args.gpus)
+    try:
+        run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,164 @@
+/*
+ * moe_b200.h -- C ABI of the routed mixture-of-experts expert forward for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operation (Hugging Face Transformers docs page "Experts backends",
+ * introduction): for each token a router selects k experts; the token's hidden
+ * state is projected through each selected expert's parameters and the expert
+ * outputs are aggregated with the routing weights. Each expert is a gated MLP
+ * (backend table, row "deepgemm_megamoe"): up projection, SwiGLU, down
+ * projection, with SwiGLU meaning silu(gate) * up (section "SonicMoE").
+ *
+ * Conventions shared by every entry point:
+ *  - All tensor pointers are DEVICE pointers owned by the caller. The library
+ *    never allocates, frees or copies between host and device, and never
+ *    synchronises the host, except where an entry point says so.
+ *  - Work is enqueued on `stream` (a cudaStream_t passed as void*; NULL is the
+ *    legacy default stream) and runs asynchronously, in stream order.
+ *  - Arguments are validated on the host before anything is enqueued; a
+ *    rejected call returns a negative moe_status and enqueues nothing.
+ *  - Errors found on the device (routing indices out of range, a bounded wait
+ *    that gave up) are recorded in the workspace's status word; read them with
+ *    moe_read_device_status.
+ *  - Layouts are row-major with the last index contiguous. bf16 is IEEE
+ *    bfloat16; e4m3 is OCP FP8 E4M3 (float8_e4m3fn); UE8M0 is an unsigned
+ *    8-bit power-of-two exponent, byte b meaning 2^(b-127).
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = -1,    /* bad shape, null pointer or misaligned pointer */
+  MOE_ERR_UNSUPPORTED = -2,    /* valid request this build does not implement */
+  MOE_ERR_SCALE_FORMAT = -3,   /* FP8 experts without UE8M0 block scales */
+  MOE_ERR_WORKSPACE = -4,      /* workspace smaller than moe_workspace_size() */
+  MOE_ERR_CUDA = -5,           /* a CUDA runtime call or launch failed */
+  MOE_ERR_DEVICE_TIMEOUT = -6, /* a kernel gave up waiting (device status) */
+  MOE_ERR_DEVICE_INDEX = -7    /* topk_idx held an index outside [0,E) or a repeated expert */
+} moe_status;
+
+/* Expert weight type. */
+typedef enum { MOE_DT_BF16 = 0, MOE_DT_E4M3 = 1 } moe_wdtype;
+
+/* Which execution of the expert matmuls to use (the page's decode-stage switch:
+ * small token counts run better on a per-token form than on grouped GEMM tiles). */
+typedef enum {
+  MOE_PATH_AUTO = 0,    /* DECODE when T*k <= 4*E and weights are bf16, else PREFILL */
+  MOE_PATH_PREFILL = 1, /* expert-major permute + tcgen05 grouped GEMMs */
+  MOE_PATH_DECODE = 2   /* weight-streaming kernels, no tile padding (bf16 only) */
+} moe_path;
+
+/* Problem shape. T tokens, hidden size H, expert intermediate size I,
+ * E experts, top-k. Requirements: T >= 0; H and I positive multiples of 128;
+ * 1 <= E <= 1024; 1 <= k <= E; T*k < 2^31 and every buffer below 2^31 rows. */
+typedef struct {
+  int32_t T, H, I, E, k;
+  int32_t wdtype; /* moe_wdtype */
+  int32_t path;   /* moe_path */
+} moe_shape;
+
+/*
+ * moe_route -- router top-k ("Experts backends", introduction: "a router
+ * selects k experts"). For each token t: softmax over the E fp32 logits, the k
+ * experts with the largest logits (equal logits: lower index first), slot j
+ * holding the j-th largest, and their probabilities renormalised to sum to 1.
+ *
+ *   logits    [T, E] fp32, finite values (a NaN logit gives an unspecified choice)
+ *   topk_idx  [T, k] int32 out
+ *   topk_w    [T, k] fp32 out
+ * Requirements: T >= 0, 1 <= E <= 1024, 1 <= k <= E. T == 0 is a no-op.
+ */
+moe_status moe_route(const float* logits, int32_t T, int32_t E, int32_t k,
+                     int32_t* topk_idx, float* topk_w, void* stream);
+
+/* Bytes of device workspace moe_forward needs for `shape` (an upper bound
+ * that depends only on the shape; host-only, enqueues nothing). Returns 0 for
+ * an invalid shape. */
+size_t moe_workspace_size(const moe_shape* shape);
+
+/*
+ * moe_forward -- the routed expert forward ("Experts backends", introduction;
+ * the "eager" row of the backend table is its reference definition):
+ *   out[t] = sum_j topk_w[t,j] * Wd[e] (silu(Wg[e] x[t]) * (Wu[e] x[t])),  e = topk_idx[t,j]
+ *
+ *   x          [T, H] bf16
+ *   topk_idx   [T, k] int32, each row k distinct experts in [0, E)
+ *   topk_w     [T, k] fp32
+ *   w_gate_up  [E, 2I, H]: rows 0..I-1 of expert e are the gate projection,
+ *              rows I..2I-1 the up projection. bf16, or e4m3 codes.
+ *   w_down     [E, H, I], bf16 or e4m3 codes.
+ *   sw_gate_up [E, 2I/128, H/128] UE8M0, one per 128x128 block (e4m3 only, else NULL)
+ *   sw_down    [E, H/128, I/128] UE8M0 (e4m3 only, else NULL)
+ *   out        [T, H] bf16 out
+ *   workspace  >= moe_workspace_size(shape) bytes, 256-byte aligned; its
+ *              previous contents do not matter. Calls that share a workspace
+ *              must not overlap in time.
+ * Intermediates: h = silu(gate) * up is rounded to bf16 and the expert output
+ * y to bf16 (e4m3 experts: x and h are quantised per token and per 128-column
+ * group with an fp32 scale amax/448, the FP8 reading of section "FP8 and FP4
+ * quantized experts"; y stays bf16). The weighted sum runs in fp32 over j in
+ * ascending order, so results are deterministic run to run.
+ * Errors: MOE_ERR_SCALE_FORMAT when wdtype is e4m3 and a scale pointer is NULL
+ * (the page's note: Blackwell kernels need UE8M0 scales and refuse plain float
+ * ones instead of silently corrupting the output); MOE_ERR_UNSUPPORTED for
+ * MOE_PATH_DECODE with e4m3 weights.
+ */
+moe_status moe_forward(const moe_shape* shape, const void* x, const int32_t* topk_idx,
+                       const float* topk_w, const void* w_gate_up, const void* w_down,
+                       const uint8_t* sw_gate_up, const uint8_t* sw_down, void* out,
+                       void* workspace, size_t workspace_bytes, void* stream);
+
+/* moe_forward that also records caller-created CUDA events (cudaEvent_t passed
+ * as void*) between its stages, on `stream`: events[0] before the permute,
+ * [1] after it, [2] after the gate/up stage, [3] after the down stage, [4]
+ * after the combine. n_events must be 5 (or 0 with events NULL). */
+moe_status moe_forward_timed(const moe_shape* shape, const void* x, const int32_t* topk_idx,
+                             const float* topk_w, const void* w_gate_up, const void* w_down,
+                             const uint8_t* sw_gate_up, const uint8_t* sw_down, void* out,
+                             void* workspace, size_t workspace_bytes, void* stream,
+                             void* const* events, int32_t n_events);
+
+/* Byte offsets, inside the workspace, of the intermediate buffers of the last
+ * moe_forward with this shape (for tests and inspection; host-only).
+ *   bm        rows per expert tile (128 for PREFILL, 1 for DECODE); path: resolved path
+ *   cnt       int32 [E]    assignments per expert
+ *   mt_base   int32 [E+1]  expert e owns rows [mt_base[e]*bm, mt_base[e+1]*bm)
+ *   row_src   int32 [m_rows] assignment t*k+j held by each row, -1 for padding
+ *   slot_row  int32 [T*k]  row of assignment t*k+j
+ *   xa        permuted activations (PREFILL): bf16 [m_rows, H] or e4m3 [m_rows, H]
+ *   xs        fp32 [m_rows, H/128] activation scales (e4m3 only)
+ *   h         bf16 [m_rows, I] (or e4m3 with fp32 scales hs [m_rows, I/128])
+ *   y         bf16 [m_rows, H] expert outputs
+ * m_rows is the allocated row capacity; only rows below mt_base[E]*bm are used.
+ * An offset of SIZE_MAX means the buffer is not used by that path. */
+typedef struct {
+  size_t status, hdr, cnt, mt_base, row_src, slot_row, xa, xs, h, hs, y, total;
+  int32_t bm, path, m_rows, reserved;
+} moe_workspace_layout;
+
+moe_status moe_workspace_query(const moe_shape* shape, moe_workspace_layout* layout);
+
+/* Synchronises `stream`, then reads the device status word the last
+ * moe_forward on this workspace wrote: MOE_OK, MOE_ERR_DEVICE_INDEX or
+ * MOE_ERR_DEVICE_TIMEOUT (MOE_ERR_CUDA if the copy itself fails). */
+moe_status moe_read_device_status(const void* workspace, void* stream);
+
+/* Static description of a status code (never NULL). */
+const char* moe_status_string(moe_status status);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int32_t moe_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

@@ -1,0 +1,195 @@
+"""Routed mixture-of-experts expert forward for NVIDIA B200 (sm_100a).
+
+Thin Python binding over the C ABI in ``include/moe_b200.h`` (library
+``libmoe_b200.so``, built in-tree by ``_build.py``). Every step of the forward
+runs in the library's CUDA kernels; this module only marshals arguments:
+torch tensors provide device memory, ``torch.cuda.current_stream()`` the
+stream. There is no CPU fallback: if the library is missing or cannot be
+loaded, every entry point raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmoe_b200.so")
+
+MOE_OK = 0
+STATUS = {
+    0: "MOE_OK", -1: "MOE_ERR_INVALID_ARG", -2: "MOE_ERR_UNSUPPORTED", -3: "MOE_ERR_SCALE_FORMAT",
+    -4: "MOE_ERR_WORKSPACE", -5: "MOE_ERR_CUDA", -6: "MOE_ERR_DEVICE_TIMEOUT", -7: "MOE_ERR_DEVICE_INDEX",
+}
+WDTYPE = {"bf16": 0, "e4m3": 1}
+PATH = {"auto": 0, "prefill": 1, "decode": 2}
+PATH_NAMES = {v: k for k, v in PATH.items()}
+EXPORTS = ["moe_route", "moe_workspace_size", "moe_forward", "moe_forward_timed", "moe_workspace_query",
+           "moe_read_device_status", "moe_status_string", "moe_version"]
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS.get(status, status)} ({status_string(status)})")
+
+
+class MoeShape(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int32), ("H", ctypes.c_int32), ("I", ctypes.c_int32), ("E", ctypes.c_int32),
+                ("k", ctypes.c_int32), ("wdtype", ctypes.c_int32), ("path", ctypes.c_int32)]
+
+
+class MoeWorkspaceLayout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in
+                ("status", "hdr", "cnt", "mt_base", "row_src", "slot_row", "xa", "xs", "h", "hs", "y", "total")] + \
+               [(n, ctypes.c_int32) for n in ("bm", "path", "m_rows", "reserved")]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded CUDA library (raises if it is missing: there is no fallback)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing; build it with "
+                              "`python -m mixture_experts_routed_moe_b200._build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+        L.moe_route.argtypes = [vp, i32, i32, i32, vp, vp, vp]
+        L.moe_route.restype = i32
+        L.moe_workspace_size.argtypes = [ctypes.POINTER(MoeShape)]
+        L.moe_workspace_size.restype = sz
+        fwd = [ctypes.POINTER(MoeShape), vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.moe_forward.argtypes = fwd
+        L.moe_forward.restype = i32
+        L.moe_forward_timed.argtypes = fwd + [ctypes.POINTER(vp), i32]
+        L.moe_forward_timed.restype = i32
+        L.moe_workspace_query.argtypes = [ctypes.POINTER(MoeShape), ctypes.POINTER(MoeWorkspaceLayout)]
+        L.moe_workspace_query.restype = i32
+        L.moe_read_device_status.argtypes = [vp, vp]
+        L.moe_read_device_status.restype = i32
+        L.moe_status_string.argtypes = [i32]
+        L.moe_status_string.restype = ctypes.c_char_p
+        L.moe_version.argtypes = []
+        L.moe_version.restype = i32
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().moe_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str):
+    if status != MOE_OK:
+        raise MoeError(status, what)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def make_shape(T, H, I, E, k, wdtype="bf16", path="auto") -> MoeShape:
+    return MoeShape(int(T), int(H), int(I), int(E), int(k), WDTYPE[wdtype] if isinstance(wdtype, str) else int(wdtype),
+                    PATH[path] if isinstance(path, str) else int(path))
+
+
+def workspace_size(shape: MoeShape) -> int:
+    n = lib().moe_workspace_size(ctypes.byref(shape))
+    if n == 0:
+        raise MoeError(-1, "moe_workspace_size")
+    return int(n)
+
+
+def workspace_layout(shape: MoeShape) -> MoeWorkspaceLayout:
+    lay = MoeWorkspaceLayout()
+    _check(lib().moe_workspace_query(ctypes.byref(shape), ctypes.byref(lay)), "moe_workspace_query")
+    return lay
+
+
+def alloc_workspace(shape: MoeShape, device=None) -> torch.Tensor:
+    """A device buffer of moe_workspace_size(shape) bytes (torch allocates it)."""
+    return torch.empty(workspace_size(shape), dtype=torch.uint8, device=device or "cuda")
+
+
+def route(logits: torch.Tensor, k: int, topk_idx: torch.Tensor | None = None, topk_w: torch.Tensor | None = None,
+          stream=None):
+    """moe_route: fp32 logits [T,E] -> (int32 [T,k], fp32 [T,k])."""
+    T, E = logits.shape
+    if topk_idx is None:
+        topk_idx = torch.empty((T, k), dtype=torch.int32, device=logits.device)
+    if topk_w is None:
+        topk_w = torch.empty((T, k), dtype=torch.float32, device=logits.device)
+    assert logits.dtype == torch.float32 and logits.is_contiguous()
+    _check(lib().moe_route(_ptr(logits), T, E, k, _ptr(topk_idx), _ptr(topk_w), _stream(stream)), "moe_route")
+    return topk_idx, topk_w
+
+
+def forward(x, topk_idx, topk_w, w_gate_up, w_down, sw_gate_up=None, sw_down=None, out=None, workspace=None,
+            path="auto", stream=None, events=None):
+    """moe_forward: bf16 x [T,H] with routing [T,k] through experts
+    w_gate_up [E,2I,H], w_down [E,H,I] (bf16, or float8_e4m3fn with uint8 UE8M0
+    block scales) -> bf16 out [T,H]. Returns (out, workspace)."""
+    T, H = x.shape
+    k = topk_idx.shape[1]
+    E, twoI, _ = w_gate_up.shape
+    wdtype = "e4m3" if w_gate_up.dtype == torch.float8_e4m3fn else "bf16"
+    shape = make_shape(T, H, twoI // 2, E, k, wdtype, path)
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device)
+    if workspace is None:
+        workspace = alloc_workspace(shape, x.device)
+    args = [ctypes.byref(shape), _ptr(x), _ptr(topk_idx), _ptr(topk_w), _ptr(w_gate_up), _ptr(w_down),
+            _ptr(sw_gate_up), _ptr(sw_down), _ptr(out), _ptr(workspace), workspace.numel(), _stream(stream)]
+    if events is None:
+        _check(lib().moe_forward(*args), "moe_forward")
+    else:
+        ev = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+        _check(lib().moe_forward_timed(*args, ev, len(events)), "moe_forward_timed")
+    return out, workspace
+
+
+def read_device_status(workspace: torch.Tensor, stream=None) -> int:
+    """Synchronises the stream and returns the device status of the last forward on `workspace`."""
+    return int(lib().moe_read_device_status(_ptr(workspace), _stream(stream)))
+
+
+class MoELayer:
+    """A routed MoE layer whose expert weights live on the GPU: ``layer(x, logits)``
+    runs moe_route then moe_forward and returns bf16 [T,H]. The workspace is
+    allocated once per shape and reused."""
+
+    def __init__(self, w_gate_up, w_down, k, sw_gate_up=None, sw_down=None, path="auto"):
+        self.w_gate_up, self.w_down = w_gate_up, w_down
+        self.sw_gate_up, self.sw_down = sw_gate_up, sw_down
+        self.k, self.path = int(k), path
+        self.E, twoI, self.H = w_gate_up.shape
+        self.I = twoI // 2
+        self._ws = {}
+
+    def _workspace(self, T, device):
+        wdtype = "e4m3" if self.w_gate_up.dtype == torch.float8_e4m3fn else "bf16"
+        shape = make_shape(T, self.H, self.I, self.E, self.k, wdtype, self.path)
+        key = (T, str(device))
+        if key not in self._ws:
+            self._ws[key] = alloc_workspace(shape, device)
+        return self._ws[key]
+
+    def __call__(self, x, logits, out=None, events=None):
+        idx, w = route(logits, self.k)
+        out, _ = forward(x, idx, w, self.w_gate_up, self.w_down, self.sw_gate_up, self.sw_down, out=out,
+                         workspace=self._workspace(x.shape[0], x.device), path=self.path, events=events)
+        return out
+
+
+__all__ = ["lib", "route", "forward", "workspace_size", "workspace_layout", "alloc_workspace",
+           "read_device_status", "make_shape", "MoELayer", "MoeError", "MoeShape", "EXPORTS", "STATUS",
+           "status_string", "PATH", "WDTYPE"]

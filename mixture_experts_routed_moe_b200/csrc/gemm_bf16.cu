@@ -1,0 +1,350 @@
+// Grouped expert GEMMs on the 5th-generation tensor cores (tcgen05 + TMEM),
+// fed by TMA. One persistent kernel serves both projections of the expert MLP
+// ("Experts backends", backend table: the expert is up projection, SwiGLU,
+// down projection; grouped_mm / deepgemm run all experts in one grouped GEMM
+// over expert-sorted tokens):
+//
+//   gate/up:  h[rows of e, n..n+127] = silu(X_e Wg_e^T) * (X_e Wu_e^T)   (SwiGLU in the epilogue)
+//   down:     y[rows of e, n..n+N-1] = h_e Wd_e^T
+//
+// Tile = (expert e, 128-row block of e's permuted rows, N-column block). The
+// tile list is only known on the device (expert counts come from routing), so
+// each CTA walks tiles blockIdx.x, blockIdx.x + gridDim.x, ... and maps a tile
+// number to (e, m, n) with the per-expert tile prefix sum. Within an expert the
+// N blocks are the outer loop and the row blocks the inner one, so CTAs that
+// run at the same time share weight tiles through L2.
+//
+// Warp roles (192 threads, one CTA per SM):
+//   warp 0      TMA producer: A tile [128 x 64] and B tile [N x 64] per stage
+//   warp 1      TMEM allocator and MMA issuer (one thread): 4 MMAs of K=16 per stage
+//   warps 2..5  epilogue: TMEM -> registers -> SwiGLU / bf16 -> global memory
+// Shared memory holds a 4-stage ring; TMEM holds two accumulators of N fp32
+// columns so the epilogue of one tile overlaps the MMAs of the next.
+// For gate/up, B stacks the 128 gate rows n..n+127 (expert rows n) over the 128
+// up rows (expert rows I+n), and one MMA with N=256 produces both halves.
+#include "moe_common.cuh"
+#include "moe_internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int kBK = 64;  // bf16 elements per 128-byte row of a stage
+constexpr int kStages = 4;
+constexpr int kThreads = 192;
+
+struct GemmParams {
+  const int* mt_base;  // [E+1] per-expert 128-row tile prefix
+  const int* cnt;      // [E]
+  int E;
+  int num_kb;             // K / 64
+  int n_tiles;            // N blocks per expert
+  int b_rows_per_expert;  // rows of one expert's B matrix
+  int b_tile_stride;      // B rows between consecutive N blocks
+  int b_second_offset;    // B rows from the first to the second 128-row half (N = 256)
+  __nv_bfloat16* out;
+  int out_ld;         // elements per output row
+  int out_tile_cols;  // output columns per tile
+  int* dev_status;
+  unsigned long long timeout_ns;
+};
+
+template <int kN>
+struct Layout {
+  static constexpr int kA = kTileM * kBK * 2;  // 16 KB
+  static constexpr int kB = kN * kBK * 2;      // 32 KB for N = 256
+  static constexpr int kStage = kA + kB;
+  static constexpr int kBarriers = 2 * kStages + 5;
+  static constexpr size_t bytes(int E) {
+    return 1024 /*alignment slack*/ + static_cast<size_t>(kStages) * kStage + kBarriers * 8 + 16 +
+           static_cast<size_t>(2 * E + 1) * 4;
+  }
+};
+
+struct TileCoord {
+  int e, m, n, row0, valid;
+};
+
+// Largest e in [0, E) with s_mt[e] <= mtile (the expert owning that tile row).
+__device__ __forceinline__ int find_expert(const int* s_mt, int E, int mtile) {
+  int lo = 0, hi = E - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (s_mt[mid] <= mtile)
+      lo = mid;
+    else
+      hi = mid - 1;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ TileCoord tile_coord(int tile, const int* s_mt, const int* s_cnt, int E, int NT) {
+  TileCoord c;
+  c.e = find_expert(s_mt, E, tile / NT);
+  const int base = s_mt[c.e];
+  const int nm = s_mt[c.e + 1] - base;
+  const int local = tile - base * NT;
+  c.n = local / nm;
+  c.m = local - c.n * nm;
+  c.row0 = (base + c.m) * kTileM;
+  c.valid = min(kTileM, s_cnt[c.e] - c.m * kTileM);
+  return c;
+}
+
+template <int kN, bool kSwiGLU>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                             const GemmParams p) {
+  using L = Layout<kN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + kStages * L::kA;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + kStages * L::kB);
+  uint64_t* empty = full + kStages;
+  uint64_t* tfull = empty + kStages;  // [2]
+  uint64_t* tempty = tfull + 2;       // [2]
+  uint64_t* drain = tempty + 2;       // [1]
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
+  int* s_mt = reinterpret_cast<int*>(s_tmem + 4);
+  int* s_cnt = s_mt + p.E + 1;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i <= p.E; i += kThreads) s_mt[i] = p.mt_base[i];
+  for (int i = threadIdx.x; i < p.E; i += kThreads) s_cnt[i] = p.cnt[i];
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 4);
+    }
+    mbar_init(drain, 1);
+    *s_abort = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(s_tmem, 2 * kN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *s_tmem;
+  const int NT = p.n_tiles;
+  const int total = s_mt[p.E] * NT;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer ----------------
+      int stage = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+        const TileCoord c = tile_coord(tile, s_mt, s_cnt, p.E, NT);
+        const int brow = c.e * p.b_rows_per_expert + c.n * p.b_tile_stride;
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          if (!mbar_wait_bounded(&empty[stage], ph ^ 1, s_abort, p.dev_status, p.timeout_ns)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[stage], L::kStage);
+          tma_load_2d(sA + stage * L::kA, &tmA, &full[stage], kb * kBK, c.row0);
+          tma_load_2d(sB + stage * L::kB, &tmB, &full[stage], kb * kBK, brow);
+          if (kN == 256)
+            tma_load_2d(sB + stage * L::kB + 128 * kBK * 2, &tmB, &full[stage], kb * kBK, brow + p.b_second_offset);
+          if (++stage == kStages) {
+            stage = 0;
+            ph ^= 1;
+          }
+        }
+      }
+      if (!ok) {
+        // let the copies already issued land before the CTA can exit
+        for (int i = 0; i < kStages; ++i) {
+          if (--stage < 0) {
+            stage = kStages - 1;
+            ph ^= 1;
+          }
+          int never = 0;
+          mbar_wait_bounded(&full[stage], ph, &never, p.dev_status, 1000000ull);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer ----------------
+      constexpr uint32_t idesc = idesc_bf16_f32(kTileM, kN);
+      int stage = 0;
+      uint32_t ph = 0;
+      int acc = 0;
+      uint32_t aph = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+        if (!mbar_wait_bounded(&tempty[acc], aph ^ 1, s_abort, p.dev_status, p.timeout_ns)) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + static_cast<uint32_t>(acc * kN);
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          if (!mbar_wait_bounded(&full[stage], ph, s_abort, p.dev_status, p.timeout_ns)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + stage * L::kA);
+          const uint32_t b0 = smem_u32(sB + stage * L::kB);
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k)
+            umma_bf16(d, sdesc_kmajor_sw128(a0 + k * 32), sdesc_kmajor_sw128(b0 + k * 32), idesc,
+                      (kb | k) != 0 ? 1u : 0u);
+          umma_commit(&empty[stage]);
+          if (++stage == kStages) {
+            stage = 0;
+            ph ^= 1;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[acc]);
+        acc ^= 1;
+        if (acc == 0) aph ^= 1;
+      }
+      // every MMA issued above has finished once this commit arrives
+      umma_commit(drain);
+      int never = 0;
+      mbar_wait_bounded(drain, 0, &never, p.dev_status, p.timeout_ns);
+    }
+  } else {
+    // ---------------- epilogue ----------------
+    const int quad = warp & 3;  // TMEM lanes 32*quad .. 32*quad+31 belong to this warp
+    const int r = quad * 32 + lane;
+    int acc = 0;
+    uint32_t aph = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      const TileCoord c = tile_coord(tile, s_mt, s_cnt, p.E, NT);
+      const bool got = mbar_wait_bounded(&tfull[acc], aph, s_abort, p.dev_status, p.timeout_ns);
+      if (!__all_sync(0xffffffffu, got)) break;
+      tc_fence_after();
+      const uint32_t tb = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * kN);
+      const bool valid = r < c.valid;
+      __nv_bfloat16* dst =
+          p.out + static_cast<size_t>(c.row0 + r) * p.out_ld + static_cast<size_t>(c.n) * p.out_tile_cols;
+      if constexpr (kSwiGLU) {
+#pragma unroll 1
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t g[32], u[32];
+          tmem_ld32(tb + cc * 32, g);
+          tmem_ld32(tb + 128 + cc * 32, u);
+          tmem_ld_wait();
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            pk[i] = pack_bf16x2(swiglu(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i])),
+                                swiglu(__uint_as_float(g[2 * i + 1]), __uint_as_float(u[2 * i + 1])));
+          if (valid) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int cc = 0; cc < kN / 32; ++cc) {
+          uint32_t v[32];
+          tmem_ld32(tb + cc * 32, v);
+          tmem_ld_wait();
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+          if (valid) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+      acc ^= 1;
+      if (acc == 0) aph ^= 1;
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 2 * kN);
+  }
+}
+
+template <int kN, bool kSwiGLU>
+cudaError_t launch_one(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmParams& gp, int grid,
+                       cudaStream_t st) {
+  const size_t smem = Layout<kN>::bytes(gp.E);
+  cudaError_t err = cudaFuncSetAttribute(grouped_gemm_bf16_kernel<kN, kSwiGLU>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (err != cudaSuccess) return err;
+  grouped_gemm_bf16_kernel<kN, kSwiGLU><<<grid, kThreads, smem, st>>>(tmA, tmB, gp);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+// which = 0: gate/up + SwiGLU (xa -> h); which = 1: down (h -> y).
+cudaError_t launch_gemm_bf16(const moe_shape* s, const Plan& p, const void* w_gate_up, const void* w_down,
+                             uint8_t* ws, int which, int num_sms, cudaStream_t st) {
+  const int H = s->H, I = s->I, E = s->E;
+  GemmParams gp{};
+  gp.mt_base = reinterpret_cast<const int*>(ws + p.mt_base);
+  gp.cnt = reinterpret_cast<const int*>(ws + p.cnt);
+  gp.E = E;
+  gp.dev_status = reinterpret_cast<int*>(ws + p.status);
+  gp.timeout_ns = kDefaultTimeoutNs;
+  // every tile count is bounded by the row capacity
+  const int max_mtiles = static_cast<int>(p.m_rows / kTileM);
+  CUtensorMap tmA, tmB;
+  if (which == 0) {
+    if (!encode_tensor_map_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws + p.xa, H, p.m_rows, kBK, kTileM) ||
+        !encode_tensor_map_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w_gate_up, H,
+                              static_cast<uint64_t>(E) * 2 * I, kBK, 128))
+      return cudaErrorInvalidValue;
+    gp.num_kb = H / kBK;
+    gp.n_tiles = I / 128;
+    gp.b_rows_per_expert = 2 * I;
+    gp.b_tile_stride = 128;
+    gp.b_second_offset = I;
+    gp.out = reinterpret_cast<__nv_bfloat16*>(ws + p.h);
+    gp.out_ld = I;
+    gp.out_tile_cols = 128;
+    const int grid = std::max(1, std::min(num_sms, max_mtiles * gp.n_tiles));
+    return launch_one<256, true>(tmA, tmB, gp, grid, st);
+  }
+  if (!encode_tensor_map_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws + p.h, I, p.m_rows, kBK, kTileM) ||
+      !encode_tensor_map_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w_down, I, static_cast<uint64_t>(E) * H, kBK,
+                            128))
+    return cudaErrorInvalidValue;
+  gp.num_kb = I / kBK;
+  gp.b_rows_per_expert = H;
+  gp.b_second_offset = 128;
+  gp.out = reinterpret_cast<__nv_bfloat16*>(ws + p.y);
+  gp.out_ld = H;
+  if (H % 256 == 0) {
+    gp.n_tiles = H / 256;
+    gp.b_tile_stride = 256;
+    gp.out_tile_cols = 256;
+    const int grid = std::max(1, std::min(num_sms, max_mtiles * gp.n_tiles));
+    return launch_one<256, false>(tmA, tmB, gp, grid, st);
+  }
+  gp.n_tiles = H / 128;
+  gp.b_tile_stride = 128;
+  gp.out_tile_cols = 128;
+  const int grid = std::max(1, std::min(num_sms, max_mtiles * gp.n_tiles));
+  return launch_one<128, false>(tmA, tmB, gp, grid, st);
+}
+
+}  // namespace moe

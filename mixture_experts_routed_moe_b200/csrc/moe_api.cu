@@ -1,0 +1,286 @@
+// C ABI of the library (declared in include/moe_b200.h): host-side argument
+// validation, the workspace plan, tensor-map encoding and the launch sequence
+//   permute -> gate/up (+SwiGLU) -> down -> combine
+// for the PREFILL (tcgen05 grouped GEMM) and DECODE (weight streaming) paths.
+#include <algorithm>
+#include <atomic>
+#include <cstring>
+#include <limits>
+
+#include "moe_common.cuh"
+#include "moe_internal.h"
+
+namespace moe {
+
+namespace {
+
+constexpr size_t kAlign = 1024;
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = []() -> EncodeTiledFn {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_sm_count[kMaxDevices];
+
+}  // namespace
+
+bool encode_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, size_t elem_bytes, const void* base,
+                          uint64_t inner, uint64_t outer, uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {inner * elem_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int device_sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 0;
+  if (dev < kMaxDevices) {
+    const int cached = g_sm_count[dev].load(std::memory_order_relaxed);
+    if (cached > 0) return cached;
+  }
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  if (dev < kMaxDevices) g_sm_count[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
+
+bool validate_shape(const moe_shape* s) {
+  if (s == nullptr) return false;
+  if (s->T < 0 || s->H < 128 || s->I < 128 || s->H % 128 != 0 || s->I % 128 != 0) return false;
+  if (s->H > 65536 || s->I > 65536) return false;
+  if (s->E < 1 || s->E > 1024 || s->k < 1 || s->k > s->E) return false;
+  if (s->wdtype != MOE_DT_BF16 && s->wdtype != MOE_DT_E4M3) return false;
+  if (s->path != MOE_PATH_AUTO && s->path != MOE_PATH_PREFILL && s->path != MOE_PATH_DECODE) return false;
+  const long long A = static_cast<long long>(s->T) * s->k;
+  const long long rows = A + static_cast<long long>(std::min<long long>(s->E, A)) * (kTileM - 1) + kTileM;
+  if (rows >= (1ll << 31) || static_cast<long long>(s->E) * 2 * s->I >= (1ll << 31) ||
+      static_cast<long long>(s->E) * s->H >= (1ll << 31))
+    return false;
+  return true;
+}
+
+int resolve_path(const moe_shape* s) {
+  if (s->path != MOE_PATH_AUTO) return s->path;
+  if (s->wdtype == MOE_DT_BF16 && static_cast<long long>(s->T) * s->k <= 4ll * s->E) return MOE_PATH_DECODE;
+  return MOE_PATH_PREFILL;
+}
+
+bool make_plan(const moe_shape* s, Plan* p) {
+  if (!validate_shape(s)) return false;
+  const long long T = s->T, H = s->H, I = s->I, E = s->E, k = s->k;
+  const long long A = T * k;
+  const bool fp8 = s->wdtype == MOE_DT_E4M3;
+  p->path = resolve_path(s);
+  p->bm = (p->path == MOE_PATH_DECODE) ? 1 : kTileM;
+  if (p->bm == 1) {
+    p->m_rows = A;
+  } else {
+    const long long rows = A + std::min(E, A) * (kTileM - 1);
+    p->m_rows = std::max<long long>(kTileM, (rows + kTileM - 1) / kTileM * kTileM);
+  }
+  p->nblk = static_cast<int>(std::max<long long>(1, (T + kPermuteTokens - 1) / kPermuteTokens));
+  const size_t none = std::numeric_limits<size_t>::max();
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + std::max<size_t>(bytes, 1), kAlign);
+    return at;
+  };
+  const size_t M = static_cast<size_t>(p->m_rows);
+  p->status = take(256);
+  p->hdr = take(256);
+  p->block_counts = take(static_cast<size_t>(p->nblk) * E * 4);
+  p->cnt = take(E * 4);
+  p->mt_base = take((E + 1) * 4);
+  p->touched = take(E * 4);
+  p->local_rank = take(std::max<long long>(A, 1) * 4);
+  p->row_src = take(std::max<size_t>(M, 1) * 4);
+  p->slot_row = take(std::max<long long>(A, 1) * 4);
+  const size_t act = fp8 ? 1 : 2;
+  p->xa = (p->path == MOE_PATH_PREFILL) ? take(M * H * act) : none;
+  p->xs = (p->path == MOE_PATH_PREFILL && fp8) ? take(M * (H / 128) * 4) : none;
+  p->h = take(M * I * act);
+  p->hs = fp8 ? take(M * (I / 128) * 4) : none;
+  p->y = take(M * H * 2);
+  p->total = off;
+  return true;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+namespace {
+
+moe_status forward_impl(const moe_shape* shape, const void* x, const int32_t* topk_idx, const float* topk_w,
+                        const void* w_gate_up, const void* w_down, const uint8_t* sw_gate_up,
+                        const uint8_t* sw_down, void* out, void* workspace, size_t workspace_bytes, void* stream,
+                        void* const* events, int32_t n_events) {
+  if (!validate_shape(shape)) return MOE_ERR_INVALID_ARG;
+  if (!(n_events == 0 || (n_events == 5 && events != nullptr))) return MOE_ERR_INVALID_ARG;
+  const bool fp8 = shape->wdtype == MOE_DT_E4M3;
+  if (fp8 && (sw_gate_up == nullptr || sw_down == nullptr)) return MOE_ERR_SCALE_FORMAT;
+  Plan plan;
+  if (!make_plan(shape, &plan)) return MOE_ERR_INVALID_ARG;
+  if (fp8 && (plan.path == MOE_PATH_DECODE || !e4m3_path_available())) return MOE_ERR_UNSUPPORTED;
+  if (shape->T == 0) return MOE_OK;
+  if (x == nullptr || topk_idx == nullptr || topk_w == nullptr || w_gate_up == nullptr || w_down == nullptr ||
+      out == nullptr || workspace == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(out, 16) || !aligned(w_gate_up, 16) || !aligned(w_down, 16) ||
+      !aligned(workspace, 256) || !aligned(topk_idx, 4) || !aligned(topk_w, 4))
+    return MOE_ERR_INVALID_ARG;
+  if (workspace_bytes < plan.total) return MOE_ERR_WORKSPACE;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const int sms = device_sm_count();
+  if (sms <= 0) return MOE_ERR_CUDA;
+  auto mark = [&](int i) -> bool {
+    return n_events == 0 || cudaEventRecord(static_cast<cudaEvent_t>(events[i]), st) == cudaSuccess;
+  };
+
+  if (!mark(0)) return MOE_ERR_CUDA;
+  if (launch_permute(shape, plan, topk_idx, x, ws, st) != cudaSuccess) return MOE_ERR_CUDA;
+  if (!mark(1)) return MOE_ERR_CUDA;
+  cudaError_t err;
+  if (plan.path == MOE_PATH_DECODE) {
+    err = launch_decode(shape, plan, x, w_gate_up, w_down, ws, 0, sms, st);
+    if (err != cudaSuccess || !mark(2)) return MOE_ERR_CUDA;
+    err = launch_decode(shape, plan, x, w_gate_up, w_down, ws, 1, sms, st);
+  } else if (!fp8) {
+    err = launch_gemm_bf16(shape, plan, w_gate_up, w_down, ws, 0, sms, st);
+    if (err != cudaSuccess || !mark(2)) return MOE_ERR_CUDA;
+    err = launch_gemm_bf16(shape, plan, w_gate_up, w_down, ws, 1, sms, st);
+  } else {
+    err = launch_gemm_e4m3(shape, plan, x, w_gate_up, w_down, sw_gate_up, sw_down, ws, 0, sms, st);
+    if (err != cudaSuccess || !mark(2)) return MOE_ERR_CUDA;
+    err = launch_gemm_e4m3(shape, plan, x, w_gate_up, w_down, sw_gate_up, sw_down, ws, 1, sms, st);
+  }
+  if (err != cudaSuccess || !mark(3)) return MOE_ERR_CUDA;
+  if (launch_combine(shape, plan, topk_w, out, ws, st) != cudaSuccess) return MOE_ERR_CUDA;
+  if (!mark(4)) return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status moe_route(const float* logits, int32_t T, int32_t E, int32_t k, int32_t* topk_idx, float* topk_w,
+                     void* stream) {
+  if (T < 0 || E < 1 || E > 1024 || k < 1 || k > E) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (logits == nullptr || topk_idx == nullptr || topk_w == nullptr) return MOE_ERR_INVALID_ARG;
+  if (!aligned(logits, 4) || !aligned(topk_idx, 4) || !aligned(topk_w, 4)) return MOE_ERR_INVALID_ARG;
+  if (static_cast<long long>(T) * k >= (1ll << 31) || static_cast<long long>(T) * E >= (1ll << 40))
+    return MOE_ERR_INVALID_ARG;
+  return launch_route(logits, T, E, k, topk_idx, topk_w, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
+}
+
+size_t moe_workspace_size(const moe_shape* shape) {
+  Plan p;
+  if (!make_plan(shape, &p)) return 0;
+  return p.total;
+}
+
+moe_status moe_forward(const moe_shape* shape, const void* x, const int32_t* topk_idx, const float* topk_w,
+                       const void* w_gate_up, const void* w_down, const uint8_t* sw_gate_up, const uint8_t* sw_down,
+                       void* out, void* workspace, size_t workspace_bytes, void* stream) {
+  return forward_impl(shape, x, topk_idx, topk_w, w_gate_up, w_down, sw_gate_up, sw_down, out, workspace,
+                      workspace_bytes, stream, nullptr, 0);
+}
+
+moe_status moe_forward_timed(const moe_shape* shape, const void* x, const int32_t* topk_idx, const float* topk_w,
+                             const void* w_gate_up, const void* w_down, const uint8_t* sw_gate_up,
+                             const uint8_t* sw_down, void* out, void* workspace, size_t workspace_bytes,
+                             void* stream, void* const* events, int32_t n_events) {
+  return forward_impl(shape, x, topk_idx, topk_w, w_gate_up, w_down, sw_gate_up, sw_down, out, workspace,
+                      workspace_bytes, stream, events, n_events);
+}
+
+moe_status moe_workspace_query(const moe_shape* shape, moe_workspace_layout* layout) {
+  if (layout == nullptr) return MOE_ERR_INVALID_ARG;
+  Plan p;
+  if (!make_plan(shape, &p)) return MOE_ERR_INVALID_ARG;
+  layout->status = p.status;
+  layout->hdr = p.hdr;
+  layout->cnt = p.cnt;
+  layout->mt_base = p.mt_base;
+  layout->row_src = p.row_src;
+  layout->slot_row = p.slot_row;
+  layout->xa = p.xa;
+  layout->xs = p.xs;
+  layout->h = p.h;
+  layout->hs = p.hs;
+  layout->y = p.y;
+  layout->total = p.total;
+  layout->bm = p.bm;
+  layout->path = p.path;
+  layout->m_rows = static_cast<int32_t>(p.m_rows);
+  layout->reserved = 0;
+  return MOE_OK;
+}
+
+moe_status moe_read_device_status(const void* workspace, void* stream) {
+  if (workspace == nullptr) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int v = 0;
+  if (cudaMemcpyAsync(&v, workspace, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
+  if (v & kDevErrTimeout) return MOE_ERR_DEVICE_TIMEOUT;
+  if (v & kDevErrIndex) return MOE_ERR_DEVICE_INDEX;
+  return MOE_OK;
+}
+
+const char* moe_status_string(moe_status status) {
+  switch (status) {
+    case MOE_OK:
+      return "ok";
+    case MOE_ERR_INVALID_ARG:
+      return "invalid argument (shape, null or misaligned pointer)";
+    case MOE_ERR_UNSUPPORTED:
+      return "unsupported combination of options";
+    case MOE_ERR_SCALE_FORMAT:
+      return "FP8 experts need UE8M0 (power-of-two) block scales";
+    case MOE_ERR_WORKSPACE:
+      return "workspace smaller than moe_workspace_size()";
+    case MOE_ERR_CUDA:
+      return "CUDA runtime error";
+    case MOE_ERR_DEVICE_TIMEOUT:
+      return "a kernel gave up on a bounded wait";
+    case MOE_ERR_DEVICE_INDEX:
+      return "routing index out of range or repeated within a token";
+  }
+  return "unknown status";
+}
+
+int32_t moe_version(void) { return 100; }
+
+}  // extern "C"

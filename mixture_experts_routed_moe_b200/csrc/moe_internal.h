@@ -1,0 +1,63 @@
+// Host-side declarations shared by the library's translation units: the
+// workspace plan and the kernel launchers. Not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/moe_b200.h"
+
+namespace moe {
+
+constexpr int kTileM = 128;        // rows per expert tile on the PREFILL path
+constexpr int kPermuteTokens = 256;  // tokens per block in the permute kernels
+constexpr int kSmallPermuteT = 256;  // T up to this uses the single-block permute
+constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;  // bounded waits give up after 2 s
+
+// Where every intermediate lives inside the caller's workspace.
+struct Plan {
+  int path;        // resolved moe_path (PREFILL or DECODE)
+  int bm;          // rows per expert tile: kTileM (PREFILL) or 1 (DECODE)
+  int64_t m_rows;  // row capacity of the permuted buffers
+  int nblk;        // permute blocks of kPermuteTokens tokens
+  size_t status, hdr, block_counts, cnt, mt_base, touched, local_rank, row_src, slot_row;
+  size_t xa, xs, h, hs, y, total;
+};
+
+// Header words written on the device by the permute stage.
+enum HdrWord { kHdrMTiles = 0, kHdrTouched = 1, kHdrRows = 2 };
+
+bool validate_shape(const moe_shape* s);
+int resolve_path(const moe_shape* s);
+bool make_plan(const moe_shape* s, Plan* p);
+
+// Launchers. Each returns the launch's cudaError_t.
+cudaError_t launch_route(const float* logits, int T, int E, int k, int* idx, float* w, cudaStream_t st);
+
+cudaError_t launch_permute(const moe_shape* s, const Plan& p, const int* topk_idx, const void* x, uint8_t* ws,
+                           cudaStream_t st);
+
+cudaError_t launch_gemm_bf16(const moe_shape* s, const Plan& p, const void* w_gate_up, const void* w_down,
+                             uint8_t* ws, int which, int num_sms, cudaStream_t st);
+
+// which = 0 also quantises the permuted activations (x -> e4m3 codes + fp32 scales).
+cudaError_t launch_gemm_e4m3(const moe_shape* s, const Plan& p, const void* x, const void* w_gate_up,
+                             const void* w_down, const uint8_t* sw_gate_up, const uint8_t* sw_down, uint8_t* ws,
+                             int which, int num_sms, cudaStream_t st);
+bool e4m3_path_available();
+
+cudaError_t launch_decode(const moe_shape* s, const Plan& p, const void* x, const void* w_gate_up,
+                          const void* w_down, uint8_t* ws, int which, int num_sms, cudaStream_t st);
+
+cudaError_t launch_combine(const moe_shape* s, const Plan& p, const float* topk_w, void* out, uint8_t* ws,
+                           cudaStream_t st);
+
+// Tensor-map encoding through the driver entry point (no link-time libcuda dependency).
+bool encode_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, size_t elem_bytes, const void* base,
+                          uint64_t inner, uint64_t outer, uint32_t box_inner, uint32_t box_outer);
+
+int device_sm_count();
+
+}  // namespace moe

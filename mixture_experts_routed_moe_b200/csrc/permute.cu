@@ -1,0 +1,280 @@
+// Expert-major permutation of the T*k assignments ("Experts backends",
+// backend table rows grouped_mm / deepgemm: tokens are sorted by their
+// selected expert so that one grouped GEMM covers every expert; the deepgemm
+// row aligns each expert's block to the GEMM tile).
+//
+// Layout produced (deterministic, independent of thread timing): expert e owns
+// rows [mt_base[e]*bm, mt_base[e+1]*bm), with mt_base the exclusive prefix sum
+// of ceil(cnt[e]/bm); inside an expert the assignments appear in ascending
+// token order; pad rows hold row_src = -1.
+//
+// The rank of assignment (t, j) inside its expert is the number of tokens
+// t' < t that chose the same expert. It is computed without any ordering
+// races: each warp of a 256-token block sets, per expert, a 32-bit mask of its
+// lanes (tokens) that chose the expert; a token's rank inside the block is the
+// population count of the masks of earlier warps plus the bits of earlier
+// lanes in its own warp, and blocks are offset by an exclusive scan of the
+// per-block counts.
+#include "moe_common.cuh"
+#include "moe_internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int kWarps = kPermuteTokens / 32;  // 8 warps, one token per thread
+
+// Phase 1 of the block-level count: per-warp expert masks in shared memory.
+// Records kDevErrIndex for an index outside [0,E) or a repeated expert.
+__device__ __forceinline__ void build_masks(uint32_t* s_mask, const int* __restrict__ idx, int t, bool active, int k,
+                                            int E, int warp, int lane, int* dev_status) {
+  if (!active) return;
+  for (int j = 0; j < k; ++j) {
+    const int e = idx[static_cast<size_t>(t) * k + j];
+    if (static_cast<unsigned>(e) < static_cast<unsigned>(E)) {
+      const uint32_t old = atomicOr(&s_mask[warp * E + e], 1u << lane);
+      if (old & (1u << lane)) atomicOr(dev_status, kDevErrIndex);
+    } else {
+      atomicOr(dev_status, kDevErrIndex);
+    }
+  }
+}
+
+__device__ __forceinline__ int rank_in_block(const uint32_t* s_mask, int e, int E, int warp, int lane) {
+  int r = 0;
+  for (int w = 0; w < warp; ++w) r += __popc(s_mask[w * E + e]);
+  return r + __popc(s_mask[warp * E + e] & ((1u << lane) - 1u));
+}
+
+__global__ void __launch_bounds__(kPermuteTokens) permute_count_kernel(const int* __restrict__ idx, int T, int k,
+                                                                       int E, int* __restrict__ block_counts,
+                                                                       int* __restrict__ local_rank,
+                                                                       int* dev_status) {
+  extern __shared__ uint32_t s_mask[];  // [kWarps][E]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < kWarps * E; i += kPermuteTokens) s_mask[i] = 0;
+  __syncthreads();
+  const int t = blockIdx.x * kPermuteTokens + threadIdx.x;
+  const bool active = t < T;
+  build_masks(s_mask, idx, t, active, k, E, warp, lane, dev_status);
+  __syncthreads();
+  if (active) {
+    for (int j = 0; j < k; ++j) {
+      const size_t a = static_cast<size_t>(t) * k + j;
+      const int e = idx[a];
+      local_rank[a] = (static_cast<unsigned>(e) < static_cast<unsigned>(E)) ? rank_in_block(s_mask, e, E, warp, lane)
+                                                                             : 0;
+    }
+  }
+  for (int e = threadIdx.x; e < E; e += kPermuteTokens) {
+    int c = 0;
+    for (int w = 0; w < kWarps; ++w) c += __popc(s_mask[w * E + e]);
+    block_counts[static_cast<size_t>(blockIdx.x) * E + e] = c;
+  }
+}
+
+// Inclusive scan of one value per thread over a block of up to 1024 threads.
+__device__ __forceinline__ int block_inclusive_scan(int v, int* s_warp) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += n;
+  }
+  if (lane == 31) s_warp[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    const int nw = (blockDim.x + 31) >> 5;
+    int w = (lane < nw) ? s_warp[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += n;
+    }
+    s_warp[lane] = w;
+  }
+  __syncthreads();
+  const int r = v + (warp > 0 ? s_warp[warp - 1] : 0);
+  __syncthreads();
+  return r;
+}
+
+// Per-expert totals (thread e), expert offsets, pad rows and the list of
+// experts that received tokens. `counts` holds per-block counts on entry and
+// per-block exclusive bases on exit. Runs as one block of 1024 threads.
+__device__ __forceinline__ void scan_experts(int* __restrict__ counts, int nblk, int E, int bm, int* __restrict__ cnt,
+                                             int* __restrict__ mt_base, int* __restrict__ touched,
+                                             int* __restrict__ hdr, int* __restrict__ row_src, int* s_warp) {
+  const int e = threadIdx.x;
+  int c = 0;
+  if (e < E) {
+    for (int b = 0; b < nblk; ++b) {
+      const int v = counts[static_cast<size_t>(b) * E + e];
+      counts[static_cast<size_t>(b) * E + e] = c;
+      c += v;
+    }
+    cnt[e] = c;
+  }
+  const int tiles = (e < E) ? (c + bm - 1) / bm : 0;
+  const int used = (e < E && c > 0) ? 1 : 0;
+  const int tiles_incl = block_inclusive_scan(tiles, s_warp);
+  const int used_incl = block_inclusive_scan(used, s_warp);
+  if (e < E) {
+    const int base = tiles_incl - tiles;
+    mt_base[e] = base;
+    if (used) touched[used_incl - 1] = e;
+    for (int r = base * bm + c; r < (base + tiles) * bm; ++r) row_src[r] = -1;
+    if (e == E - 1) {
+      mt_base[E] = tiles_incl;
+      hdr[kHdrMTiles] = tiles_incl;
+      hdr[kHdrTouched] = used_incl;
+      hdr[kHdrRows] = tiles_incl * bm;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(1024) permute_scan_kernel(int* counts, int nblk, int E, int bm, int* cnt,
+                                                            int* mt_base, int* touched, int* hdr, int* row_src) {
+  __shared__ int s_warp[32];
+  scan_experts(counts, nblk, E, bm, cnt, mt_base, touched, hdr, row_src, s_warp);
+}
+
+// Copy one assignment's bf16 hidden-state row into its permuted row (one warp).
+__device__ __forceinline__ void copy_row_bf16(const __nv_bfloat16* __restrict__ x, __nv_bfloat16* __restrict__ xa,
+                                              int t, int row, int H, int lane) {
+  const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H);
+  uint4* dst = reinterpret_cast<uint4*>(xa + static_cast<size_t>(row) * H);
+  for (int c = lane; c < H / 8; c += 32) dst[c] = __ldg(src + c);
+}
+
+// One warp per assignment: writes row_src / slot_row and, when xa is given,
+// copies the token's hidden state into the permuted row.
+__global__ void __launch_bounds__(256) permute_scatter_kernel(const int* __restrict__ idx, int T, int k, int E, int bm,
+                                                              const int* __restrict__ block_base,
+                                                              const int* __restrict__ local_rank,
+                                                              const int* __restrict__ mt_base,
+                                                              int* __restrict__ row_src, int* __restrict__ slot_row,
+                                                              const __nv_bfloat16* __restrict__ x,
+                                                              __nv_bfloat16* __restrict__ xa, int H) {
+  const int lane = threadIdx.x & 31;
+  const long long a = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (a >= static_cast<long long>(T) * k) return;
+  const int t = static_cast<int>(a / k);
+  const int e = idx[a];
+  if (static_cast<unsigned>(e) >= static_cast<unsigned>(E)) {
+    if (lane == 0) slot_row[a] = -1;
+    return;
+  }
+  const int b = t / kPermuteTokens;
+  const int row = mt_base[e] * bm + block_base[static_cast<size_t>(b) * E + e] + local_rank[a];
+  if (lane == 0) {
+    row_src[row] = static_cast<int>(a);
+    slot_row[a] = row;
+  }
+  if (xa != nullptr) copy_row_bf16(x, xa, t, row, H, lane);
+}
+
+// Everything in one block of 1024 threads, for T <= kPermuteTokens.
+__global__ void __launch_bounds__(1024) permute_small_kernel(const int* __restrict__ idx, int T, int k, int E, int bm,
+                                                             int* __restrict__ cnt, int* __restrict__ mt_base,
+                                                             int* __restrict__ touched, int* __restrict__ hdr,
+                                                             int* __restrict__ row_src, int* __restrict__ slot_row,
+                                                             int* __restrict__ local_rank, int* dev_status,
+                                                             const __nv_bfloat16* __restrict__ x,
+                                                             __nv_bfloat16* __restrict__ xa, int H) {
+  extern __shared__ uint32_t s_mask[];  // [kWarps][E]
+  __shared__ int s_warp[32];
+  __shared__ int s_base[1024];  // per-expert block base is always 0 here; holds mt_base*bm
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < kWarps * E; i += blockDim.x) s_mask[i] = 0;
+  __syncthreads();
+  const int t = threadIdx.x;
+  const bool active = t < T;  // T <= 256: warps 0..7 hold the tokens
+  build_masks(s_mask, idx, t, active, k, E, warp, lane, dev_status);
+  __syncthreads();
+  if (active) {
+    for (int j = 0; j < k; ++j) {
+      const int a = t * k + j;
+      const int e = idx[a];
+      local_rank[a] = (static_cast<unsigned>(e) < static_cast<unsigned>(E)) ? rank_in_block(s_mask, e, E, warp, lane)
+                                                                             : 0;
+    }
+  }
+  // per-expert totals from the masks
+  int c = 0;
+  if (threadIdx.x < E)
+    for (int w = 0; w < kWarps; ++w) c += __popc(s_mask[w * E + threadIdx.x]);
+  const int e = threadIdx.x;
+  const int tiles = (e < E) ? (c + bm - 1) / bm : 0;
+  const int used = (e < E && c > 0) ? 1 : 0;
+  const int tiles_incl = block_inclusive_scan(tiles, s_warp);
+  const int used_incl = block_inclusive_scan(used, s_warp);
+  if (e < E) {
+    const int base = tiles_incl - tiles;
+    cnt[e] = c;
+    mt_base[e] = base;
+    s_base[e] = base * bm;
+    if (used) touched[used_incl - 1] = e;
+    for (int r = base * bm + c; r < (base + tiles) * bm; ++r) row_src[r] = -1;
+    if (e == E - 1) {
+      mt_base[E] = tiles_incl;
+      hdr[kHdrMTiles] = tiles_incl;
+      hdr[kHdrTouched] = used_incl;
+      hdr[kHdrRows] = tiles_incl * bm;
+    }
+  }
+  __syncthreads();
+  // scatter: one warp per assignment
+  for (int a = warp; a < T * k; a += 32) {
+    const int e2 = idx[a];
+    if (static_cast<unsigned>(e2) >= static_cast<unsigned>(E)) {
+      if (lane == 0) slot_row[a] = -1;
+      continue;
+    }
+    const int row = s_base[e2] + local_rank[a];
+    if (lane == 0) {
+      row_src[row] = a;
+      slot_row[a] = row;
+    }
+    if (xa != nullptr) copy_row_bf16(x, xa, a / k, row, H, lane);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_permute(const moe_shape* s, const Plan& p, const int* topk_idx, const void* x, uint8_t* ws,
+                           cudaStream_t st) {
+  const int T = s->T, k = s->k, E = s->E, H = s->H;
+  int* status = reinterpret_cast<int*>(ws + p.status);
+  int* hdr = reinterpret_cast<int*>(ws + p.hdr);
+  int* counts = reinterpret_cast<int*>(ws + p.block_counts);
+  int* cnt = reinterpret_cast<int*>(ws + p.cnt);
+  int* mt_base = reinterpret_cast<int*>(ws + p.mt_base);
+  int* touched = reinterpret_cast<int*>(ws + p.touched);
+  int* lrank = reinterpret_cast<int*>(ws + p.local_rank);
+  int* row_src = reinterpret_cast<int*>(ws + p.row_src);
+  int* slot_row = reinterpret_cast<int*>(ws + p.slot_row);
+  // the permuted bf16 copy of x is only needed by the bf16 PREFILL path
+  __nv_bfloat16* xa = (p.path == MOE_PATH_PREFILL && s->wdtype == MOE_DT_BF16)
+                          ? reinterpret_cast<__nv_bfloat16*>(ws + p.xa)
+                          : nullptr;
+  const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+  const size_t mask_bytes = sizeof(uint32_t) * kWarps * E;
+
+  cudaError_t err = cudaMemsetAsync(status, 0, sizeof(int), st);
+  if (err != cudaSuccess) return err;
+  if (T <= kSmallPermuteT) {
+    permute_small_kernel<<<1, 1024, mask_bytes, st>>>(topk_idx, T, k, E, p.bm, cnt, mt_base, touched, hdr, row_src,
+                                                      slot_row, lrank, status, xb, xa, H);
+    return cudaGetLastError();
+  }
+  permute_count_kernel<<<p.nblk, kPermuteTokens, mask_bytes, st>>>(topk_idx, T, k, E, counts, lrank, status);
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  permute_scan_kernel<<<1, 1024, 0, st>>>(counts, p.nblk, E, p.bm, cnt, mt_base, touched, hdr, row_src);
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  const long long A = static_cast<long long>(T) * k;
+  permute_scatter_kernel<<<static_cast<unsigned>((A + 7) / 8), 256, 0, st>>>(
+      topk_idx, T, k, E, p.bm, counts, lrank, mt_base, row_src, slot_row, xb, xa, H);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

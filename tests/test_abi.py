@@ -1,0 +1,131 @@
+"""The C-ABI library loads, exports every entry point the header declares, and
+rejects bad arguments on the host before touching a GPU (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import mixture_experts_routed_moe_b200 as moe
+from mixture_experts_routed_moe_b200 import _build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+FAKE = 1 << 20  # a 256-byte aligned non-null address; never dereferenced by the host checks
+
+
+@pytest.fixture(scope="module")
+def L():
+    _build.build()
+    return moe.lib()
+
+
+def header_functions():
+    text = open(os.path.join(ROOT, "include", "moe_b200.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = header_functions()
+    assert set(names) == set(moe.EXPORTS)
+    for n in names:
+        assert hasattr(L, n), n
+    nm = os.popen(f"nm -D --defined-only {moe.LIB_PATH}").read()
+    for n in names:
+        assert re.search(rf"\bT {n}\b", nm), n
+
+
+def test_version_and_status_strings(L):
+    assert L.moe_version() >= 100
+    for code in moe.STATUS:
+        assert moe.status_string(code)
+    assert "UE8M0" in moe.status_string(-3)
+
+
+def shape(**kw):
+    d = dict(T=64, H=128, I=256, E=8, k=2, wdtype="bf16", path="auto")
+    d.update(kw)
+    return moe.make_shape(**d)
+
+
+@pytest.mark.parametrize("bad", [dict(H=100), dict(I=64), dict(E=0), dict(E=1025), dict(k=0), dict(k=9),
+                                 dict(T=-1), dict(wdtype=7), dict(path=9), dict(H=0)])
+def test_invalid_shapes_rejected(L, bad):
+    s = shape(**bad)
+    assert L.moe_workspace_size(ctypes.byref(s)) == 0
+    lay = moe.MoeWorkspaceLayout()
+    assert L.moe_workspace_query(ctypes.byref(s), ctypes.byref(lay)) == -1
+    r = L.moe_forward(ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, FAKE, None, None, FAKE, FAKE, 1 << 40, None)
+    assert r == -1
+
+
+def test_workspace_layout_is_consistent(L):
+    for path, bm in (("prefill", 128), ("decode", 1)):
+        s = shape(T=300, E=60, k=4, H=2048, I=1408, path=path)
+        lay = moe.workspace_layout(s)
+        assert lay.bm == bm and lay.path == moe.PATH[path]
+        total = moe.workspace_size(s)
+        assert total == lay.total
+        A = 300 * 4
+        assert lay.m_rows >= A + (min(60, A) * (bm - 1) if bm > 1 else 0)
+        offs = [lay.status, lay.hdr, lay.cnt, lay.mt_base, lay.row_src, lay.slot_row, lay.h, lay.y]
+        assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
+        assert lay.y + lay.m_rows * 2048 * 2 <= total
+        assert (lay.xa == 2 ** 64 - 1) == (path == "decode")
+
+
+def test_auto_path_choice(L):
+    assert moe.workspace_layout(shape(T=16, H=2048, I=1408, E=60, k=4)).path == moe.PATH["decode"]
+    assert moe.workspace_layout(shape(T=8192, H=2048, I=768, E=128, k=8)).path == moe.PATH["prefill"]
+    assert moe.workspace_layout(shape(T=16, E=60, k=4, wdtype="e4m3")).path == moe.PATH["prefill"]
+
+
+def test_scale_format_error_and_host_errors(L):
+    s = shape(wdtype="e4m3")
+    # FP8 experts without UE8M0 scales: refused loudly
+    r = L.moe_forward(ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, FAKE, None, None, FAKE, FAKE, 1 << 40, None)
+    assert r == -3
+    s = shape(wdtype="e4m3", path="decode")
+    r = L.moe_forward(ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 40, None)
+    assert r == -2
+    s = shape()
+    need = moe.workspace_size(s)
+    r = L.moe_forward(ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, FAKE, None, None, FAKE, FAKE, need - 1, None)
+    assert r == -4
+    r = L.moe_forward(ctypes.byref(s), None, FAKE, FAKE, FAKE, FAKE, None, None, FAKE, FAKE, need, None)
+    assert r == -1
+    r = L.moe_forward(ctypes.byref(s), FAKE + 8, FAKE, FAKE, FAKE, FAKE, None, None, FAKE, FAKE, need, None)
+    assert r == -1  # misaligned x
+    r = L.moe_forward(ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, FAKE, None, None, FAKE, FAKE + 16, need, None)
+    assert r == -1  # misaligned workspace
+    # empty input: nothing to do, nothing enqueued
+    s0 = shape(T=0)
+    assert L.moe_forward(ctypes.byref(s0), None, None, None, None, None, None, None, None, None, 0, None) == 0
+    # bad timing-event count
+    ev = (ctypes.c_void_p * 3)()
+    assert L.moe_forward_timed(ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, FAKE, None, None, FAKE, FAKE, need, None,
+                               ev, 3) == -1
+
+
+def test_route_host_errors(L):
+    assert L.moe_route(FAKE, 4, 0, 1, FAKE, FAKE, None) == -1
+    assert L.moe_route(FAKE, 4, 8, 9, FAKE, FAKE, None) == -1
+    assert L.moe_route(FAKE, -1, 8, 2, FAKE, FAKE, None) == -1
+    assert L.moe_route(None, 4, 8, 2, FAKE, FAKE, None) == -1
+    assert L.moe_route(None, 0, 8, 2, None, None, None) == 0
+
+
+def test_missing_library_fails_loudly(monkeypatch):
+    monkeypatch.setattr(moe, "_lib", None)
+    monkeypatch.setattr(moe, "LIB_PATH", "/nonexistent/libmoe_b200.so")
+    with pytest.raises(ImportError):
+        moe.lib()
+
+
+def test_product_code_never_touches_the_oracle():
+    pkg = os.path.join(ROOT, "mixture_experts_routed_moe_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                src = open(os.path.join(dirpath, f)).read()
+                assert not re.search(r"^\s*(from|import)\s+oracle|moe_oracle|oracle/", src, flags=re.M), f

@@ -1,0 +1,161 @@
+"""moe_forward on the GPU against the oracle: permutation bit-exact, expert
+intermediates and outputs within the bf16 tolerances, on both paths, at sizes
+spanning many tiles and ragged tails, plus edge cases and the full-size
+workloads on sampled tokens."""
+import numpy as np
+import pytest
+import torch
+
+import mixture_experts_routed_moe_b200 as moe
+from mixture_experts_routed_moe_b200 import inputs as G
+from oracle import moe_oracle as O
+
+from parity import (ExpertView, assert_bf16_close, check_permutation, device_inputs, oracle_forward_bf16,
+                    ws_bf16)
+
+pytestmark = pytest.mark.gpu
+
+
+def _forward(wl, seed, path, idx=None, w=None, logits=None):
+    x, L, W = device_inputs(wl, seed)
+    if idx is None:
+        idx, w, _ = O.route(L.numpy(), wl.k)
+    else:
+        idx, w = idx.numpy(), w.numpy()
+    out, ws = moe.forward(x.cuda(), torch.from_numpy(idx).cuda(), torch.from_numpy(w).cuda(), W["w_gate_up"],
+                          W["w_down"], path=path)
+    torch.cuda.synchronize()
+    assert moe.read_device_status(ws) == 0
+    return x, idx, w, W, out, ws
+
+
+@pytest.mark.parametrize("path", ["prefill", "decode"])
+@pytest.mark.parametrize("name", ["tiny", "decode"])
+def test_small_workloads_full_parity(name, path):
+    wl = G.WORKLOADS[name]
+    x, idx, w, W, out, ws = _forward(wl, G.default_seed(wl), path)
+    shape = moe.make_shape(wl.T, wl.H, wl.I, wl.E, wl.k, "bf16", path)
+    lay, perm = check_permutation(ws, shape, idx)
+    ref = oracle_forward_bf16(x, idx, w, W)
+    assert_bf16_close(out.float().cpu().numpy(), ref, f"{name}/{path}")
+    # expert intermediates h and y for every valid row
+    rows = np.nonzero(perm["row_src"] >= 0)[0]
+    h = ws_bf16(ws, lay.h, lay.m_rows, wl.I)[rows]
+    y = ws_bf16(ws, lay.y, lay.m_rows, wl.H)[rows]
+    a = perm["row_src"][rows]
+    xr = x.float().numpy()[a // wl.k]
+    e_of = idx.ravel()[a]
+    href = np.zeros_like(h, dtype=np.float64)
+    yref = np.zeros_like(y, dtype=np.float64)
+    V1, V2 = ExpertView(W["w_gate_up"]), ExpertView(W["w_down"])
+    for e in np.unique(e_of):
+        sel = e_of == e
+        href[sel], yref[sel] = O.expert_mlp(xr[sel].astype(np.float64), V1[e], V2[e], "bf16")
+    assert_bf16_close(h, href, "h")
+    assert_bf16_close(y, yref, "y")
+
+
+@pytest.mark.parametrize("path", ["prefill", "decode"])
+def test_paths_agree_and_are_deterministic(path):
+    wl = G.Workload("mid", 300, 256, 384, 16, 4)
+    x, idx, w, W, out1, ws = _forward(wl, 11, path)
+    out2, _ = moe.forward(x.cuda(), torch.from_numpy(idx).cuda(), torch.from_numpy(w).cuda(), W["w_gate_up"],
+                          W["w_down"], path=path, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(out1, out2)  # run-to-run bit identical
+    check_permutation(ws, moe.make_shape(wl.T, wl.H, wl.I, wl.E, wl.k, "bf16", path), idx)
+    ref = oracle_forward_bf16(x, idx, w, W)
+    assert_bf16_close(out1.float().cpu().numpy(), ref, path)
+
+
+EDGE_COUNTS = [
+    # (T, H, I, E, k, counts): empty experts, 1, BM-1, BM, BM+1, 2*BM-1, 2*BM rows
+    (896, 256, 256, 8, 1, [0, 1, 127, 128, 129, 255, 256, 0]),
+    (300, 128, 256, 4, 1, [300, 0, 0, 0]),  # every token on one expert
+    (200, 128, 128, 3, 2, [200, 200, 0]),
+    (1, 256, 128, 8, 8, [1] * 8),  # one token, k = E
+    (257, 128, 128, 5, 3, [257, 257, 257, 0, 0]),  # just above the single-block permute
+    (256, 128, 128, 5, 3, [256, 256, 256, 0, 0]),  # at it
+    (16, 2048, 1408, 4, 2, [16, 16, 0, 0]),  # decode token groups beyond 4
+]
+
+
+@pytest.mark.parametrize("path", ["prefill", "decode"])
+@pytest.mark.parametrize("T,H,I,E,k,counts", EDGE_COUNTS)
+def test_edge_counts(T, H, I, E, k, counts, path):
+    wl = G.Workload("edge", T, H, I, E, k)
+    idx, w = G.routed_inputs_with_counts(wl, counts, seed=T)
+    x, idx_np, w_np, W, out, ws = _forward(wl, 3, path, idx=idx, w=w)
+    check_permutation(ws, moe.make_shape(T, H, I, E, k, "bf16", path), idx_np)
+    ref = oracle_forward_bf16(x, idx_np, w_np, W)
+    assert_bf16_close(out.float().cpu().numpy(), ref, f"edge {counts} {path}")
+
+
+def test_many_experts_random_routing():
+    wl = G.Workload("wide", 512, 256, 256, 1024, 8)
+    x, idx, w, W, out, ws = _forward(wl, 5, "prefill")
+    check_permutation(ws, moe.make_shape(wl.T, wl.H, wl.I, wl.E, wl.k, "bf16", "prefill"), idx)
+    assert_bf16_close(out.float().cpu().numpy(), oracle_forward_bf16(x, idx, w, W), "wide")
+
+
+def test_end_to_end_with_gpu_routing():
+    """GPU route -> GPU forward against oracle route -> oracle forward."""
+    wl = G.WORKLOADS["tiny"]
+    x, L, W = device_inputs(wl, 0)
+    layer = moe.MoELayer(W["w_gate_up"], W["w_down"], wl.k)
+    out = layer(x.cuda(), L.cuda())
+    idx, w, _ = O.route(L.numpy(), wl.k)
+    assert_bf16_close(out.float().cpu().numpy(), oracle_forward_bf16(x, idx, w, W), "e2e")
+
+
+def test_bad_routing_index_is_reported_not_faulted():
+    wl = G.Workload("bad", 40, 128, 128, 4, 2)
+    x, L, W = device_inputs(wl, 1)
+    idx, w, _ = O.route(L.numpy(), wl.k)
+    idx = idx.copy()
+    idx[3, 1] = 4  # out of range
+    idx[7, 1] = idx[7, 0]  # repeated expert
+    for path in ("prefill", "decode"):
+        out, ws = moe.forward(x.cuda(), torch.from_numpy(idx).cuda(), torch.from_numpy(w).cuda(), W["w_gate_up"],
+                              W["w_down"], path=path)
+        assert moe.read_device_status(ws) == -7
+    # the next good call on the same workspace clears the status
+    idx2, w2, _ = O.route(L.numpy(), wl.k)
+    moe.forward(x.cuda(), torch.from_numpy(idx2).cuda(), torch.from_numpy(w2).cuda(), W["w_gate_up"], W["w_down"],
+                workspace=ws, path="decode")
+    assert moe.read_device_status(ws) == 0
+
+
+def test_empty_input():
+    wl = G.Workload("empty", 0, 128, 128, 4, 2)
+    W = G.make_weights(wl, 0, device="cuda")
+    x = torch.empty((0, 128), dtype=torch.bfloat16, device="cuda")
+    out, _ = moe.forward(x, torch.empty((0, 2), dtype=torch.int32, device="cuda"),
+                         torch.empty((0, 2), dtype=torch.float32, device="cuda"), W["w_gate_up"], W["w_down"])
+    assert out.shape == (0, 128)
+
+
+SAMPLE = np.array([0, 1, 2, 3, 5, 8, 13, 100, 511, 1000, 2047, 3001, 4094, 4095])
+
+
+@pytest.mark.parametrize("name", ["prefill", "skewed"])
+def test_full_size_bf16_sampled(name):
+    """Full-size workload in the launch configuration the benchmark times
+    (AUTO path); the oracle computes a sample of tokens one by one, and the
+    permutation is checked in full."""
+    wl = G.WORKLOADS[name]
+    seed = G.default_seed(wl)
+    x, L, W = device_inputs(wl, seed)
+    layer = moe.MoELayer(W["w_gate_up"], W["w_down"], wl.k)
+    out = layer(x.cuda(), L.cuda())
+    torch.cuda.synchronize()
+    idx, w, _ = O.route(L.numpy(), wl.k)
+    ws = layer._workspace(wl.T, x.cuda().device)
+    assert moe.read_device_status(ws) == 0
+    check_permutation(ws, moe.make_shape(wl.T, wl.H, wl.I, wl.E, wl.k, "bf16", "auto"), idx)
+    toks = np.concatenate([SAMPLE[SAMPLE < wl.T], [wl.T - 1]])
+    ref = oracle_forward_bf16(x, idx, w, W, tokens=toks)
+    assert_bf16_close(out.float().cpu().numpy()[toks], ref, name)
+    # every output row is finite and non-trivial
+    o = out.float()
+    assert torch.isfinite(o).all() and (o.abs().amax(dim=1) > 0).all()
