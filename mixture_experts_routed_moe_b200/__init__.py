@@ -152,6 +152,9 @@ def forward(x, topk_idx, topk_w, w_gate_up, w_down, sw_gate_up=None, sw_down=Non
     if events is None:
         _check(lib().moe_forward(*args), "moe_forward")
     else:
+        for e in events:  # torch creates the CUDA event lazily, on its first record
+            if not e.cuda_event:
+                e.record(stream or torch.cuda.current_stream())
         ev = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
         _check(lib().moe_forward_timed(*args, ev, len(events)), "moe_forward_timed")
     return out, workspace

@@ -49,7 +49,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) route_kernel(const float*
   for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
 
   uint32_t taken = 0;  // bit i: expert lane + 32*i already selected
-  float psum = 0.f;
+  float psum = 0.f, pcomp = 0.f;  // compensated (Kahan) sum of the chosen probabilities
   int* idx_out = topk_idx + static_cast<size_t>(t) * k;
   float* w_out = topk_w + static_cast<size_t>(t) * k;
   for (int j = 0; j < k; ++j) {
@@ -75,7 +75,10 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) route_kernel(const float*
     // the owner lane marks the winner as taken
     if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
     const float p = expf(bv - vmax) / z;  // softmax probability of the winner
-    psum += p;
+    const float yk = p - pcomp;
+    const float tk = psum + yk;
+    pcomp = (tk - psum) - yk;
+    psum = tk;
     if (lane == 0) {
       idx_out[j] = bi;
       w_out[j] = p;
