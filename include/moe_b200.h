@@ -42,7 +42,8 @@ typedef enum {
   MOE_ERR_WORKSPACE = -4,      /* workspace smaller than moe_workspace_size() */
   MOE_ERR_CUDA = -5,           /* a CUDA runtime call or launch failed */
   MOE_ERR_DEVICE_TIMEOUT = -6, /* a kernel gave up waiting (device status) */
-  MOE_ERR_DEVICE_INDEX = -7    /* topk_idx held an index outside [0,E) or a repeated expert */
+  MOE_ERR_DEVICE_INDEX = -7,   /* topk_idx held an index outside [0,E) or a repeated expert */
+  MOE_ERR_SCRATCH_LIMIT = -8   /* moe_forward_noalloc: the shape needs more scratch than the library holds */
 } moe_status;
 
 /* Expert weight type. */
@@ -150,6 +151,30 @@ moe_status moe_workspace_query(const moe_shape* shape, moe_workspace_layout* lay
  * moe_forward on this workspace wrote: MOE_OK, MOE_ERR_DEVICE_INDEX or
  * MOE_ERR_DEVICE_TIMEOUT (MOE_ERR_CUDA if the copy itself fails). */
 moe_status moe_read_device_status(const void* workspace, void* stream);
+
+/*
+ * moe_forward_noalloc -- moe_forward for callers that cannot allocate device
+ * memory. The page has no counterpart to this entry point; it exists for
+ * callers that are handed only their input and output buffers (a plugin loaded
+ * by a host framework that gives it no allocator) and for latency-critical
+ * paths that must not call cudaMalloc, which can synchronise the device.
+ *
+ * Arguments and results are those of moe_forward, without the workspace: the
+ * scratch space lives in a fixed array of MOE_NOALLOC_SCRATCH_BYTES bytes in
+ * the library's own device memory (every GPU that loads the library holds it
+ * until the process exits). Nothing is allocated or freed.
+ *  - A shape whose moe_workspace_size() exceeds MOE_NOALLOC_SCRATCH_BYTES is
+ *    rejected with MOE_ERR_SCRATCH_LIMIT before anything is enqueued.
+ *  - The first call on each device looks up the array's device address (with
+ *    that device current); make that first call before any stream capture.
+ *  - All calls share the one array and leave their intermediates in it. Calls
+ *    whose GPU work overlaps in time race on it: order them, for example by
+ *    issuing them on one stream. moe_read_device_status does not apply here.
+ */
+#define MOE_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20) /* 8 MiB */
+moe_status moe_forward_noalloc(const moe_shape* shape, const void* x, const int32_t* topk_idx,
+                               const float* topk_w, const void* w_gate_up, const void* w_down,
+                               const uint8_t* sw_gate_up, const uint8_t* sw_down, void* out, void* stream);
 
 /* Static description of a status code (never NULL). */
 const char* moe_status_string(moe_status status);

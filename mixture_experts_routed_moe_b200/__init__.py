@@ -21,12 +21,13 @@ MOE_OK = 0
 STATUS = {
     0: "MOE_OK", -1: "MOE_ERR_INVALID_ARG", -2: "MOE_ERR_UNSUPPORTED", -3: "MOE_ERR_SCALE_FORMAT",
     -4: "MOE_ERR_WORKSPACE", -5: "MOE_ERR_CUDA", -6: "MOE_ERR_DEVICE_TIMEOUT", -7: "MOE_ERR_DEVICE_INDEX",
+    -8: "MOE_ERR_SCRATCH_LIMIT",
 }
 WDTYPE = {"bf16": 0, "e4m3": 1}
 PATH = {"auto": 0, "prefill": 1, "decode": 2}
 PATH_NAMES = {v: k for k, v in PATH.items()}
 EXPORTS = ["moe_route", "moe_workspace_size", "moe_forward", "moe_forward_timed", "moe_workspace_query",
-           "moe_read_device_status", "moe_status_string", "moe_version"]
+           "moe_read_device_status", "moe_status_string", "moe_version", "moe_forward_noalloc"]
 
 
 class MoeError(RuntimeError):
@@ -73,6 +74,8 @@ def lib() -> ctypes.CDLL:
         L.moe_read_device_status.restype = i32
         L.moe_status_string.argtypes = [i32]
         L.moe_status_string.restype = ctypes.c_char_p
+        L.moe_forward_noalloc.argtypes = [ctypes.POINTER(MoeShape), vp, vp, vp, vp, vp, vp, vp, vp, vp]
+        L.moe_forward_noalloc.restype = i32
         L.moe_version.argtypes = []
         L.moe_version.restype = i32
         _lib = L
@@ -160,6 +163,25 @@ def forward(x, topk_idx, topk_w, w_gate_up, w_down, sw_gate_up=None, sw_down=Non
     return out, workspace
 
 
+def forward_noalloc(x, topk_idx, topk_w, w_gate_up, w_down, sw_gate_up=None, sw_down=None, out=None, path="auto",
+                    stream=None):
+    """moe_forward_noalloc: the forward with the library's own fixed scratch
+    array instead of a caller workspace, for callers that cannot allocate device
+    memory (only ``out`` is allocated here when not given). Calls share the
+    array, so calls whose GPU work overlaps must be ordered by the caller."""
+    T, H = x.shape
+    k = topk_idx.shape[1]
+    E, twoI, _ = w_gate_up.shape
+    wdtype = "e4m3" if w_gate_up.dtype == torch.float8_e4m3fn else "bf16"
+    shape = make_shape(T, H, twoI // 2, E, k, wdtype, path)
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device)
+    _check(lib().moe_forward_noalloc(ctypes.byref(shape), _ptr(x), _ptr(topk_idx), _ptr(topk_w), _ptr(w_gate_up),
+                                     _ptr(w_down), _ptr(sw_gate_up), _ptr(sw_down), _ptr(out), _stream(stream)),
+           "moe_forward_noalloc")
+    return out
+
+
 def read_device_status(workspace: torch.Tensor, stream=None) -> int:
     """Synchronises the stream and returns the device status of the last forward on `workspace`."""
     return int(lib().moe_read_device_status(_ptr(workspace), _stream(stream)))
@@ -193,6 +215,6 @@ class MoELayer:
         return out
 
 
-__all__ = ["lib", "route", "forward", "workspace_size", "workspace_layout", "alloc_workspace",
+__all__ = ["lib", "route", "forward", "forward_noalloc", "workspace_size", "workspace_layout", "alloc_workspace",
            "read_device_status", "make_shape", "MoELayer", "MoeError", "MoeShape", "EXPORTS", "STATUS",
            "status_string", "PATH", "WDTYPE"]

@@ -277,6 +277,8 @@ const char* moe_status_string(moe_status status) {
       return "a kernel gave up on a bounded wait";
     case MOE_ERR_DEVICE_INDEX:
       return "routing index out of range or repeated within a token";
+    case MOE_ERR_SCRATCH_LIMIT:
+      return "shape needs more scratch than the allocation-free entry point holds";
   }
   return "unknown status";
 }
