@@ -356,8 +356,6 @@ def run_ours(args, world, rank, local):
 
     peaks, peak_src = load_peaks()
     per_step_launches = 1 + (1 if wl.T <= 256 else 3) + 2 + 1  # route, permute, gate/up, down, combine
-    if wl.wdtype == "e4m3":
-        per_step_launches += 1  # activation quantisation
     tokens = wl.T * K * world
     value = tokens / (total_ms / 1e3)
     line = {

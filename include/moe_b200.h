@@ -110,7 +110,8 @@ size_t moe_workspace_size(const moe_shape* shape);
  * Errors: MOE_ERR_SCALE_FORMAT when wdtype is e4m3 and a scale pointer is NULL
  * (the page's note: Blackwell kernels need UE8M0 scales and refuse plain float
  * ones instead of silently corrupting the output); MOE_ERR_UNSUPPORTED for
- * MOE_PATH_DECODE with e4m3 weights.
+ * MOE_PATH_DECODE with e4m3 weights and for e4m3 weights with H not a multiple
+ * of 256.
  */
 moe_status moe_forward(const moe_shape* shape, const void* x, const int32_t* topk_idx,
                        const float* topk_w, const void* w_gate_up, const void* w_down,

@@ -24,6 +24,7 @@
 // up rows (expert rows I+n), and one MMA with N=256 produces both halves.
 #include "moe_common.cuh"
 #include "moe_internal.h"
+#include "tile_sched.cuh"
 
 namespace moe {
 namespace {
@@ -59,36 +60,6 @@ struct Layout {
            static_cast<size_t>(2 * E + 1) * 4;
   }
 };
-
-struct TileCoord {
-  int e, m, n, row0, valid;
-};
-
-// Largest e in [0, E) with s_mt[e] <= mtile (the expert owning that tile row).
-__device__ __forceinline__ int find_expert(const int* s_mt, int E, int mtile) {
-  int lo = 0, hi = E - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (s_mt[mid] <= mtile)
-      lo = mid;
-    else
-      hi = mid - 1;
-  }
-  return lo;
-}
-
-__device__ __forceinline__ TileCoord tile_coord(int tile, const int* s_mt, const int* s_cnt, int E, int NT) {
-  TileCoord c;
-  c.e = find_expert(s_mt, E, tile / NT);
-  const int base = s_mt[c.e];
-  const int nm = s_mt[c.e + 1] - base;
-  const int local = tile - base * NT;
-  c.n = local / nm;
-  c.m = local - c.n * nm;
-  c.row0 = (base + c.m) * kTileM;
-  c.valid = min(kTileM, s_cnt[c.e] - c.m * kTileM);
-  return c;
-}
 
 template <int kN, bool kSwiGLU>
 __global__ void __launch_bounds__(kThreads, 1)

@@ -1,13 +1,367 @@
-// FP8 (e4m3) expert GEMMs: not built yet.
+// FP8 (e4m3) expert GEMMs on tcgen05 (kind::f8f6f4), fed by TMA ("Experts
+// backends", section "FP8 and FP4 quantized experts": FP8 experts with
+// dynamic per-row activation scales; on Blackwell the expert weight scales are
+// UE8M0 powers of two, one per 128x128 block).
+//
+//   gate/up:  h = silu(Xg) * Xu with X = q_x * s_x (per row, per 128 columns) and
+//             W = q_w * 2^(b-127) (per 128x128 block); h is quantised again per
+//             row and 128 columns (e4m3 codes + fp32 scale)
+//   down:     y = h W_d^T, rounded to bf16
+//
+// The activation scales are arbitrary fp32 numbers, so they cannot ride in the
+// MMA's UE8M0 block scales. Instead every 128-wide K block goes through the
+// tensor core on its own: 4 MMAs of K=32 write a fresh fp32 partial into one of
+// two TMEM buffers, and 8 epilogue warps read it back and promote it into
+// register accumulators with the combined scale s_x[row, kb] * 2^(b[nb, kb]-127).
+// While they promote one partial, the tensor core fills the other.
+//
+// Warp roles (320 threads, one CTA per SM): warp 0 TMA producer, warp 1 TMEM
+// allocator and MMA issuer, warps 2..9 promotion + epilogue. Warps w and w+4
+// share TMEM lane quadrant w%4 (rows); warp group 2..5 takes the first half of
+// each 128-column block pair, 6..9 the second. Tiles and their order are those
+// of the bf16 kernel (tile_sched.cuh).
+#include "moe_common.cuh"
 #include "moe_internal.h"
+#include "tile_sched.cuh"
 
 namespace moe {
+namespace {
 
-bool e4m3_path_available() { return false; }
+constexpr int kBK = 128;  // e4m3 elements per 128-byte stage row = one scale block
+constexpr int kStages = 4;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr int kA = kTileM * kBK;  // 16 KB
+constexpr int kB = 256 * kBK;     // 32 KB
+constexpr int kStage = kA + kB;
+constexpr int kBarriers = 2 * kStages + 5;
 
-cudaError_t launch_gemm_e4m3(const moe_shape*, const Plan&, const void*, const void*, const void*, const uint8_t*,
-                             const uint8_t*, uint8_t*, int, int, cudaStream_t) {
-  return cudaErrorNotSupported;
+size_t smem_bytes(int E) {
+  return 1024 + static_cast<size_t>(kStages) * kStage + kBarriers * 8 + 16 + 2 * kTileM * 4 +
+         static_cast<size_t>(2 * E + 1) * 4;
+}
+
+struct Fp8Params {
+  const int* mt_base;
+  const int* cnt;
+  int E;
+  int num_kb;             // K / 128
+  int n_tiles;            // column blocks per expert
+  int b_rows_per_expert;  // rows of one expert's B matrix
+  int b_tile_stride;      // B rows between consecutive column blocks
+  int b_second_offset;    // B rows from the first 128-row half to the second
+  const float* a_scale;   // [m_rows, num_kb]
+  const uint8_t* w_scale; // [E, b_rows_per_expert/128, num_kb]
+  uint8_t* hq;            // gate/up: e4m3 h [m_rows, I]
+  float* hs;              // gate/up: h scales [m_rows, I/128]
+  __nv_bfloat16* y;       // down: [m_rows, H]
+  int out_ld;             // I (gate/up) or H (down)
+  int* dev_status;
+  unsigned long long timeout_ns;
+};
+
+__device__ __forceinline__ float ue8m0_value(uint32_t b) {
+  if (b == 0) return 5.877471754111438e-39f;  // 2^-127 (subnormal)
+  if (b == 255) return __int_as_float(0x7fc00000);
+  return __int_as_float(b << 23);
+}
+
+__device__ __forceinline__ void epi_bar_sync() { asm volatile("bar.sync 1, %0;" ::"n"(32 * kEpiWarps) : "memory"); }
+
+template <bool kGateUp>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemm_e4m3_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                             const Fp8Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + kStages * kA;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + kStages * kB);
+  uint64_t* empty = full + kStages;
+  uint64_t* pfull = empty + kStages;  // [2] partial accumulator ready
+  uint64_t* pempty = pfull + 2;       // [2] partial accumulator consumed
+  uint64_t* drain = pempty + 2;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
+  float* s_amax = reinterpret_cast<float*>(s_tmem + 4);  // [2][128]
+  int* s_mt = reinterpret_cast<int*>(s_amax + 2 * kTileM);
+  int* s_cnt = s_mt + p.E + 1;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i <= p.E; i += kThreads) s_mt[i] = p.mt_base[i];
+  for (int i = threadIdx.x; i < p.E; i += kThreads) s_cnt[i] = p.cnt[i];
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&pfull[b], 1);
+      mbar_init(&pempty[b], kEpiWarps);
+    }
+    mbar_init(drain, 1);
+    *s_abort = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(s_tmem, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *s_tmem;
+  const int NT = p.n_tiles;
+  const int KB = p.num_kb;
+  const int total = s_mt[p.E] * NT;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer ----------------
+      int stage = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+        const TileCoord c = tile_coord(tile, s_mt, s_cnt, p.E, NT);
+        const int brow = c.e * p.b_rows_per_expert + c.n * p.b_tile_stride;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait_bounded(&empty[stage], ph ^ 1, s_abort, p.dev_status, p.timeout_ns)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[stage], kStage);
+          tma_load_2d(sA + stage * kA, &tmA, &full[stage], kb * kBK, c.row0);
+          tma_load_2d(sB + stage * kB, &tmB, &full[stage], kb * kBK, brow);
+          tma_load_2d(sB + stage * kB + 128 * kBK, &tmB, &full[stage], kb * kBK, brow + p.b_second_offset);
+          if (++stage == kStages) {
+            stage = 0;
+            ph ^= 1;
+          }
+        }
+      }
+      if (!ok) {
+        for (int i = 0; i < kStages; ++i) {
+          if (--stage < 0) {
+            stage = kStages - 1;
+            ph ^= 1;
+          }
+          int never = 0;
+          mbar_wait_bounded(&full[stage], ph, &never, p.dev_status, 1000000ull);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer: one fresh partial per 128-wide K block ----------------
+      constexpr uint32_t idesc = idesc_e4m3_f32(kTileM, 256);
+      int stage = 0, pb = 0;
+      uint32_t ph = 0, pph = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait_bounded(&full[stage], ph, s_abort, p.dev_status, p.timeout_ns) ||
+              !mbar_wait_bounded(&pempty[pb], pph ^ 1, s_abort, p.dev_status, p.timeout_ns)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t d = tmem_base + static_cast<uint32_t>(pb * 256);
+          const uint32_t a0 = smem_u32(sA + stage * kA);
+          const uint32_t b0 = smem_u32(sB + stage * kB);
+#pragma unroll
+          for (int k = 0; k < kBK / 32; ++k)
+            umma_e4m3(d, sdesc_kmajor_sw128(a0 + k * 32), sdesc_kmajor_sw128(b0 + k * 32), idesc, k != 0 ? 1u : 0u);
+          umma_commit(&empty[stage]);
+          umma_commit(&pfull[pb]);
+          if (++stage == kStages) {
+            stage = 0;
+            ph ^= 1;
+          }
+          pb ^= 1;
+          if (pb == 0) pph ^= 1;
+        }
+      }
+      umma_commit(drain);
+      int never = 0;
+      mbar_wait_bounded(drain, 0, &never, p.dev_status, p.timeout_ns);
+    }
+  } else {
+    // ---------------- promotion + epilogue ----------------
+    const int quad = warp & 3;
+    const int hf = (warp - 2) >> 2;  // 0: warps 2..5, 1: warps 6..9
+    const int r = quad * 32 + lane;
+    const int wrows = p.b_rows_per_expert / 128;  // weight scale rows per expert
+    int pb = 0;
+    uint32_t pph = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+      const TileCoord c = tile_coord(tile, s_mt, s_cnt, p.E, NT);
+      const int row = c.row0 + r;
+      // weight scale rows of the two 128-column halves this thread promotes
+      int nb0, nb1;
+      if (kGateUp) {
+        nb0 = c.n;                                 // gate block
+        nb1 = p.b_second_offset / 128 + c.n;       // up block
+      } else {
+        nb0 = nb1 = 2 * c.n + hf;
+      }
+      const uint8_t* ws0 = p.w_scale + (static_cast<size_t>(c.e) * wrows + nb0) * KB;
+      const uint8_t* ws1 = p.w_scale + (static_cast<size_t>(c.e) * wrows + nb1) * KB;
+      const float* xsr = p.a_scale + static_cast<size_t>(row) * KB;
+      float acc[128];
+#pragma unroll
+      for (int i = 0; i < 128; ++i) acc[i] = 0.f;
+      float sx_next = __ldg(xsr);
+      for (int kb = 0; kb < KB; ++kb) {
+        const float sx = sx_next;
+        if (kb + 1 < KB) sx_next = __ldg(xsr + kb + 1);
+        const float sc0 = sx * ue8m0_value(__ldg(ws0 + kb));
+        const float sc1 = sx * ue8m0_value(__ldg(ws1 + kb));
+        const bool got = mbar_wait_bounded(&pfull[pb], pph, s_abort, p.dev_status, p.timeout_ns);
+        if (!__all_sync(0xffffffffu, got)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t tb = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(pb * 256);
+        // gate/up: columns [64hf, 64hf+64) of the gate half and the same of the up half;
+        // down: columns [128hf, 128hf+128)
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const uint32_t col = kGateUp ? ((q < 4 ? 0u : 128u) + 64u * hf + 16u * (q & 3)) : (128u * hf + 16u * q);
+          uint32_t v[16];
+          tmem_ld16(tb + col, v);
+          tmem_ld_wait();
+          const float sc = (kGateUp && q >= 4) ? sc1 : sc0;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) acc[16 * q + i] = fmaf(__uint_as_float(v[i]), sc, acc[16 * q + i]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&pempty[pb]);
+        pb ^= 1;
+        if (pb == 0) pph ^= 1;
+      }
+      if (!ok) break;
+      // a warp that gave up on a wait raised the abort flag before leaving; never
+      // enter the named barrier below without it
+      if (__any_sync(0xffffffffu, *s_abort != 0)) break;
+      const bool valid = r < c.valid;
+      if constexpr (kGateUp) {
+        // h for columns n*128 + 64hf + i, i < 64: acc[i] is the gate, acc[64+i] the up projection
+        float amax = 0.f;
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          acc[i] = swiglu(acc[i], acc[64 + i]);
+          amax = fmaxf(amax, fabsf(acc[i]));
+        }
+        s_amax[hf * kTileM + r] = amax;
+        epi_bar_sync();
+        amax = fmaxf(s_amax[r], s_amax[kTileM + r]);
+        epi_bar_sync();
+        const float sc = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+        if (valid) {
+          uint32_t w[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const uint32_t lo = __nv_cvt_float2_to_fp8x2(
+                make_float2(__fdiv_rn(acc[4 * i], sc), __fdiv_rn(acc[4 * i + 1], sc)), __NV_SATFINITE, __NV_E4M3);
+            const uint32_t hi = __nv_cvt_float2_to_fp8x2(
+                make_float2(__fdiv_rn(acc[4 * i + 2], sc), __fdiv_rn(acc[4 * i + 3], sc)), __NV_SATFINITE, __NV_E4M3);
+            w[i] = lo | (hi << 16);
+          }
+          uint4* dst = reinterpret_cast<uint4*>(p.hq + static_cast<size_t>(row) * p.out_ld + c.n * 128 + hf * 64);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+          if (hf == 0) p.hs[static_cast<size_t>(row) * (p.out_ld / 128) + c.n] = sc;
+        }
+      } else {
+        if (valid) {
+          uint4* dst = reinterpret_cast<uint4*>(p.y + static_cast<size_t>(row) * p.out_ld + c.n * 256 + hf * 128);
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            dst[i] = make_uint4(pack_bf16x2(acc[8 * i], acc[8 * i + 1]), pack_bf16x2(acc[8 * i + 2], acc[8 * i + 3]),
+                                pack_bf16x2(acc[8 * i + 4], acc[8 * i + 5]),
+                                pack_bf16x2(acc[8 * i + 6], acc[8 * i + 7]));
+        }
+      }
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+template <bool kGateUp>
+cudaError_t launch_one(const CUtensorMap& tmA, const CUtensorMap& tmB, const Fp8Params& fp, int grid,
+                       cudaStream_t st) {
+  const size_t smem = smem_bytes(fp.E);
+  cudaError_t err = cudaFuncSetAttribute(grouped_gemm_e4m3_kernel<kGateUp>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (err != cudaSuccess) return err;
+  grouped_gemm_e4m3_kernel<kGateUp><<<grid, kThreads, smem, st>>>(tmA, tmB, fp);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool e4m3_path_available() { return true; }
+
+// which = 0: gate/up (+SwiGLU, h quantised); which = 1: down. The activation
+// quantisation of x happens in the permute stage.
+cudaError_t launch_gemm_e4m3(const moe_shape* s, const Plan& p, const void* /*x*/, const void* w_gate_up,
+                             const void* w_down, const uint8_t* sw_gate_up, const uint8_t* sw_down, uint8_t* ws,
+                             int which, int num_sms, cudaStream_t st) {
+  const int H = s->H, I = s->I, E = s->E;
+  Fp8Params fp{};
+  fp.mt_base = reinterpret_cast<const int*>(ws + p.mt_base);
+  fp.cnt = reinterpret_cast<const int*>(ws + p.cnt);
+  fp.E = E;
+  fp.dev_status = reinterpret_cast<int*>(ws + p.status);
+  fp.timeout_ns = kDefaultTimeoutNs;
+  const int max_mtiles = static_cast<int>(p.m_rows / kTileM);
+  CUtensorMap tmA, tmB;
+  if (which == 0) {
+    if (!encode_tensor_map_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ws + p.xa, H, p.m_rows, kBK, kTileM) ||
+        !encode_tensor_map_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w_gate_up, H, static_cast<uint64_t>(E) * 2 * I,
+                              kBK, 128))
+      return cudaErrorInvalidValue;
+    fp.num_kb = H / kBK;
+    fp.n_tiles = I / 128;
+    fp.b_rows_per_expert = 2 * I;
+    fp.b_tile_stride = 128;
+    fp.b_second_offset = I;
+    fp.a_scale = reinterpret_cast<const float*>(ws + p.xs);
+    fp.w_scale = sw_gate_up;
+    fp.hq = ws + p.h;
+    fp.hs = reinterpret_cast<float*>(ws + p.hs);
+    fp.out_ld = I;
+    const int grid = std::max(1, std::min(num_sms, max_mtiles * fp.n_tiles));
+    return launch_one<true>(tmA, tmB, fp, grid, st);
+  }
+  if (H % 256 != 0) return cudaErrorNotSupported;  // the down tile spans two 128-column scale blocks
+  if (!encode_tensor_map_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ws + p.h, I, p.m_rows, kBK, kTileM) ||
+      !encode_tensor_map_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w_down, I, static_cast<uint64_t>(E) * H, kBK,
+                            128))
+    return cudaErrorInvalidValue;
+  fp.num_kb = I / kBK;
+  fp.n_tiles = H / 256;
+  fp.b_rows_per_expert = H;
+  fp.b_tile_stride = 256;
+  fp.b_second_offset = 128;
+  fp.a_scale = reinterpret_cast<const float*>(ws + p.hs);
+  fp.w_scale = sw_down;
+  fp.y = reinterpret_cast<__nv_bfloat16*>(ws + p.y);
+  fp.out_ld = H;
+  const int grid = std::max(1, std::min(num_sms, max_mtiles * fp.n_tiles));
+  return launch_one<false>(tmA, tmB, fp, grid, st);
 }
 
 }  // namespace moe

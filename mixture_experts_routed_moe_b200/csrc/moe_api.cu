@@ -146,7 +146,9 @@ moe_status forward_impl(const moe_shape* shape, const void* x, const int32_t* to
   if (fp8 && (sw_gate_up == nullptr || sw_down == nullptr)) return MOE_ERR_SCALE_FORMAT;
   Plan plan;
   if (!make_plan(shape, &plan)) return MOE_ERR_INVALID_ARG;
-  if (fp8 && (plan.path == MOE_PATH_DECODE || !e4m3_path_available())) return MOE_ERR_UNSUPPORTED;
+  // e4m3 experts: PREFILL only, and the down tile spans two 128-column scale blocks
+  if (fp8 && (plan.path == MOE_PATH_DECODE || !e4m3_path_available() || shape->H % 256 != 0))
+    return MOE_ERR_UNSUPPORTED;
   if (shape->T == 0) return MOE_OK;
   if (x == nullptr || topk_idx == nullptr || topk_w == nullptr || w_gate_up == nullptr || w_down == nullptr ||
       out == nullptr || workspace == nullptr)

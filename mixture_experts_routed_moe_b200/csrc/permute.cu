@@ -146,15 +146,51 @@ __device__ __forceinline__ void copy_row_bf16(const __nv_bfloat16* __restrict__ 
   for (int c = lane; c < H / 8; c += 32) dst[c] = __ldg(src + c);
 }
 
+// Quantise one assignment's hidden-state row into its permuted row (one warp):
+// per 128-column group, scale s = amax/448 in fp32 (1 for an all-zero group)
+// and codes e4m3(x/s), round to nearest even, saturating (the FP8 experts'
+// dynamic per-row activation scales). Each half-warp owns one group at a time.
+__device__ __forceinline__ void quant_row_e4m3(const __nv_bfloat16* __restrict__ x, uint8_t* __restrict__ xq,
+                                               float* __restrict__ xs, int t, int row, int H, int lane) {
+  const int half = lane >> 4, l16 = lane & 15;
+  const unsigned hmask = 0xFFFFu << (16 * half);
+  const int G = H / 128;
+  const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H);
+  for (int g = half; g < G; g += 2) {
+    const uint4 v = __ldg(src + g * 16 + l16);
+    const float f[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
+                        bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(hmask, amax, o));
+    const float sc = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+    uint32_t w[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(__fdiv_rn(f[4 * i], sc), __fdiv_rn(f[4 * i + 1], sc)),
+                                                   __NV_SATFINITE, __NV_E4M3);
+      const uint32_t hi = __nv_cvt_float2_to_fp8x2(
+          make_float2(__fdiv_rn(f[4 * i + 2], sc), __fdiv_rn(f[4 * i + 3], sc)), __NV_SATFINITE, __NV_E4M3);
+      w[i] = lo | (hi << 16);
+    }
+    *reinterpret_cast<uint2*>(xq + static_cast<size_t>(row) * H + g * 128 + l16 * 8) = make_uint2(w[0], w[1]);
+    if (l16 == 0) xs[static_cast<size_t>(row) * G + g] = sc;
+  }
+}
+
 // One warp per assignment: writes row_src / slot_row and, when xa is given,
-// copies the token's hidden state into the permuted row.
+// copies the token's hidden state into the permuted row (or, when xq is given,
+// quantises it to e4m3 with per-group scales in xs).
 __global__ void __launch_bounds__(256) permute_scatter_kernel(const int* __restrict__ idx, int T, int k, int E, int bm,
                                                               const int* __restrict__ block_base,
                                                               const int* __restrict__ local_rank,
                                                               const int* __restrict__ mt_base,
                                                               int* __restrict__ row_src, int* __restrict__ slot_row,
                                                               const __nv_bfloat16* __restrict__ x,
-                                                              __nv_bfloat16* __restrict__ xa, int H) {
+                                                              __nv_bfloat16* __restrict__ xa, uint8_t* __restrict__ xq,
+                                                              float* __restrict__ xs, int H) {
   const int lane = threadIdx.x & 31;
   const long long a = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   if (a >= static_cast<long long>(T) * k) return;
@@ -171,6 +207,7 @@ __global__ void __launch_bounds__(256) permute_scatter_kernel(const int* __restr
     slot_row[a] = row;
   }
   if (xa != nullptr) copy_row_bf16(x, xa, t, row, H, lane);
+  if (xq != nullptr) quant_row_e4m3(x, xq, xs, t, row, H, lane);
 }
 
 // Everything in one block of 1024 threads, for T <= kPermuteTokens.
@@ -180,7 +217,8 @@ __global__ void __launch_bounds__(1024) permute_small_kernel(const int* __restri
                                                              int* __restrict__ row_src, int* __restrict__ slot_row,
                                                              int* __restrict__ local_rank, int* dev_status,
                                                              const __nv_bfloat16* __restrict__ x,
-                                                             __nv_bfloat16* __restrict__ xa, int H) {
+                                                             __nv_bfloat16* __restrict__ xa, uint8_t* __restrict__ xq,
+                                                             float* __restrict__ xs, int H) {
   extern __shared__ uint32_t s_mask[];  // [kWarps][E]
   __shared__ int s_warp[32];
   __shared__ int s_base[1024];  // per-expert block base is always 0 here; holds mt_base*bm
@@ -236,6 +274,7 @@ __global__ void __launch_bounds__(1024) permute_small_kernel(const int* __restri
       slot_row[a] = row;
     }
     if (xa != nullptr) copy_row_bf16(x, xa, a / k, row, H, lane);
+    if (xq != nullptr) quant_row_e4m3(x, xq, xs, a / k, row, H, lane);
   }
 }
 
@@ -257,6 +296,9 @@ cudaError_t launch_permute(const moe_shape* s, const Plan& p, const int* topk_id
   __nv_bfloat16* xa = (p.path == MOE_PATH_PREFILL && s->wdtype == MOE_DT_BF16)
                           ? reinterpret_cast<__nv_bfloat16*>(ws + p.xa)
                           : nullptr;
+  // the e4m3 PREFILL path quantises x into its permuted rows instead
+  uint8_t* xq = (p.path == MOE_PATH_PREFILL && s->wdtype == MOE_DT_E4M3) ? ws + p.xa : nullptr;
+  float* xs = xq != nullptr ? reinterpret_cast<float*>(ws + p.xs) : nullptr;
   const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
   const size_t mask_bytes = sizeof(uint32_t) * kWarps * E;
 
@@ -264,7 +306,7 @@ cudaError_t launch_permute(const moe_shape* s, const Plan& p, const int* topk_id
   if (err != cudaSuccess) return err;
   if (T <= kSmallPermuteT) {
     permute_small_kernel<<<1, 1024, mask_bytes, st>>>(topk_idx, T, k, E, p.bm, cnt, mt_base, touched, hdr, row_src,
-                                                      slot_row, lrank, status, xb, xa, H);
+                                                      slot_row, lrank, status, xb, xa, xq, xs, H);
     return cudaGetLastError();
   }
   permute_count_kernel<<<p.nblk, kPermuteTokens, mask_bytes, st>>>(topk_idx, T, k, E, counts, lrank, status);
@@ -273,7 +315,7 @@ cudaError_t launch_permute(const moe_shape* s, const Plan& p, const int* topk_id
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   const long long A = static_cast<long long>(T) * k;
   permute_scatter_kernel<<<static_cast<unsigned>((A + 7) / 8), 256, 0, st>>>(
-      topk_idx, T, k, E, p.bm, counts, lrank, mt_base, row_src, slot_row, xb, xa, H);
+      topk_idx, T, k, E, p.bm, counts, lrank, mt_base, row_src, slot_row, xb, xa, xq, xs, H);
   return cudaGetLastError();
 }
 
