@@ -218,7 +218,13 @@ def oracle_sample_rate(wl, seed, n_tokens, steps=1, warmup=0):
 
 
 def oracle_sample_tokens(wl):
-    return min(wl.T, 16)
+    """Tokens per oracle sample, sized for roughly 10-30 s of CPU work: the
+    eager loop's cost is dominated by converting each touched expert's weights
+    to float64 (dequantising them for e4m3), about 3*H*I elements per expert."""
+    per_expert = 3 * wl.H * wl.I * (4 if wl.wdtype == "e4m3" else 1)
+    budget = 3.0e9  # element conversions
+    experts = max(1, int(budget // per_expert))
+    return max(1, min(wl.T, 16, experts // wl.k))
 
 
 def run_reference(args, world, rank):
