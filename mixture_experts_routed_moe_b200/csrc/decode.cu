@@ -6,9 +6,10 @@
 // With only a few tokens per expert, the layer is bound by reading each
 // touched expert's weights once from HBM. Every warp owns a few consecutive
 // weight rows of one touched expert, streams them with 16-byte no-L1 loads and
-// dots them against all of that expert's tokens (kept in L1/L2). No tile
-// padding, no tensor cores: the FMAs are far below the CUDA-core peak at these
-// token counts.
+// dots them against all of that expert's tokens (kept in L1/L2), converting
+// each weight chunk to fp32 once for all tokens. No tile padding, no tensor
+// cores: the work is bound by HBM. The grid is exactly one wave of resident
+// blocks.
 //
 //   gate/up:  h[row, n] = silu(<x_t, Wg_e[n]>) * <x_t, Wu_e[n]>  (bf16)
 //   down:     y[row, c] = <h[row], Wd_e[c]>                      (bf16)
@@ -23,25 +24,69 @@ namespace {
 constexpr int kBlock = 256;
 constexpr int kWarpsPerBlock = kBlock / 32;
 
-// Reduce 32 per-lane partial sums across the warp with 31 shuffles; afterwards
-// lane l holds the full sum of value index l.
-__device__ __forceinline__ float warp_transpose_reduce(float (&v)[32], int lane) {
-#pragma unroll
-  for (int s = 16; s >= 1; s >>= 1) {
-    const bool upper = (lane & s) != 0;
-#pragma unroll
-    for (int i = 0; i < s; ++i) {
-      const float send = upper ? v[i] : v[i + s];
-      const float keep = upper ? v[i + s] : v[i];
-      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, s);
-    }
-  }
-  return v[0];
+__device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
+  f[0] = bf16_lo(v.x);
+  f[1] = bf16_hi(v.x);
+  f[2] = bf16_lo(v.y);
+  f[3] = bf16_hi(v.y);
+  f[4] = bf16_lo(v.z);
+  f[5] = bf16_hi(v.z);
+  f[6] = bf16_lo(v.w);
+  f[7] = bf16_hi(v.w);
 }
 
-// gate/up: a task is (touched expert u, 4 consecutive rows n0..n0+3 of I, a
-// group of up to 4 of the expert's tokens). Value index (0..31) =
-// half*16 + row*4 + token, half 0 = gate, 1 = up.
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// acc[r][q] += <weight row r, activation row q> over this lane's 16-byte
+// chunks (NR rows, NQ activation rows). All NR weight loads of a chunk step
+// are issued together; each weight chunk is converted to fp32 once and each
+// activation chunk once, then shared by every (row, token) pair.
+template <int NR, int NQ>
+__device__ __forceinline__ void dot_rows(const __nv_bfloat16* const (&w)[NR], const __nv_bfloat16* const (&a)[4],
+                                         int nch, int lane, float (&acc)[NR][4]) {
+  for (int ch = lane; ch < nch; ch += 32) {
+    uint4 wv[NR];
+#pragma unroll
+    for (int r = 0; r < NR; ++r) wv[r] = ld_stream_u4(w[r] + ch * 8);
+    float xf[NQ][8];
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) unpack8(__ldg(reinterpret_cast<const uint4*>(a[q]) + ch), xf[q]);
+#pragma unroll
+    for (int r = 0; r < NR; ++r) {
+      float wf[8];
+      unpack8(wv[r], wf);
+#pragma unroll
+      for (int q = 0; q < NQ; ++q)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[r][q] = fmaf(wf[i], xf[q][i], acc[r][q]);
+    }
+  }
+}
+
+// gate/up: a task is (touched expert u, 4 consecutive rows n0..n0+3 of I);
+// weight rows 0..3 are gate rows n0.., rows 4..7 the up rows I+n0...
+template <int NQ>
+__device__ __forceinline__ void gate_up_group(const __nv_bfloat16* const (&w)[8], const __nv_bfloat16* const (&a)[4],
+                                              int nch, int lane, __nv_bfloat16* h, size_t row0, int I, int n0) {
+  float acc[8][4];
+#pragma unroll
+  for (int r = 0; r < 8; ++r)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) acc[r][q] = 0.f;
+  dot_rows<8, NQ>(w, a, nch, lane, acc);
+#pragma unroll
+  for (int q = 0; q < NQ; ++q)
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const float g = warp_sum(acc[r][q]), u = warp_sum(acc[4 + r][q]);
+      if (lane == r) h[(row0 + q) * I + n0 + r] = __float2bfloat16_rn(swiglu(g, u));
+    }
+}
+
 __global__ void __launch_bounds__(kBlock) decode_gate_up_kernel(
     const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ wgu, const int* __restrict__ cnt,
     const int* __restrict__ row_off, const int* __restrict__ row_src, const int* __restrict__ touched,
@@ -60,47 +105,47 @@ __global__ void __launch_bounds__(kBlock) decode_gate_up_kernel(
     const int c_e = cnt[e];
     const int r_e = row_off[e];
     const __nv_bfloat16* wg = wgu + (static_cast<size_t>(e) * 2 * I + n0) * H;
-    const __nv_bfloat16* wu = wg + static_cast<size_t>(I) * H;
+    const __nv_bfloat16* w[8];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      w[r] = wg + static_cast<size_t>(r) * H;
+      w[4 + r] = wg + (static_cast<size_t>(I) + r) * H;
+    }
     for (int g0 = 0; g0 < c_e; g0 += 4) {
       const int ntok = min(4, c_e - g0);
-      const __nv_bfloat16* xt[4];
+      const __nv_bfloat16* a[4];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int rr = r_e + g0 + min(q, ntok - 1);
-        xt[q] = x + static_cast<size_t>(row_src[rr] / k) * H;
-      }
-      float acc[32];
-#pragma unroll
-      for (int i = 0; i < 32; ++i) acc[i] = 0.f;
-      for (int ch = lane; ch < nch; ch += 32) {
-        uint4 a[4], b[4], xv[4];
-#pragma unroll
-        for (int rw = 0; rw < 4; ++rw) {
-          a[rw] = ld_stream_u4(wg + static_cast<size_t>(rw) * H + ch * 8);
-          b[rw] = ld_stream_u4(wu + static_cast<size_t>(rw) * H + ch * 8);
-        }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) xv[q] = __ldg(reinterpret_cast<const uint4*>(xt[q]) + ch);
-#pragma unroll
-        for (int rw = 0; rw < 4; ++rw)
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            acc[rw * 4 + q] = dot8_bf16(a[rw], xv[q], acc[rw * 4 + q]);
-            acc[16 + rw * 4 + q] = dot8_bf16(b[rw], xv[q], acc[16 + rw * 4 + q]);
-          }
-      }
-      const float sum = warp_transpose_reduce(acc, lane);
-      const float up = __shfl_down_sync(0xffffffffu, sum, 16);
-      if (lane < 16) {
-        const int rw = lane >> 2, q = lane & 3;
-        if (q < ntok) h[static_cast<size_t>(r_e + g0 + q) * I + n0 + rw] = __float2bfloat16_rn(swiglu(sum, up));
+      for (int q = 0; q < 4; ++q) a[q] = x + static_cast<size_t>(row_src[r_e + g0 + min(q, ntok - 1)] / k) * H;
+      const size_t row0 = static_cast<size_t>(r_e + g0);
+      switch (ntok) {
+        case 1: gate_up_group<1>(w, a, nch, lane, h, row0, I, n0); break;
+        case 2: gate_up_group<2>(w, a, nch, lane, h, row0, I, n0); break;
+        case 3: gate_up_group<3>(w, a, nch, lane, h, row0, I, n0); break;
+        default: gate_up_group<4>(w, a, nch, lane, h, row0, I, n0); break;
       }
     }
   }
 }
 
-// down: a task is (touched expert u, 8 consecutive rows c0..c0+7 of H, a group
-// of up to 4 tokens). Value index = row*4 + token.
+// down: a task is (touched expert u, 8 consecutive rows c0..c0+7 of H).
+template <int NQ>
+__device__ __forceinline__ void down_group(const __nv_bfloat16* const (&w)[8], const __nv_bfloat16* const (&a)[4],
+                                           int nch, int lane, __nv_bfloat16* y, size_t row0, int H, int c0) {
+  float acc[8][4];
+#pragma unroll
+  for (int r = 0; r < 8; ++r)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) acc[r][q] = 0.f;
+  dot_rows<8, NQ>(w, a, nch, lane, acc);
+#pragma unroll
+  for (int q = 0; q < NQ; ++q)
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const float v = warp_sum(acc[r][q]);
+      if (lane == r) y[(row0 + q) * H + c0 + r] = __float2bfloat16_rn(v);
+    }
+}
+
 __global__ void __launch_bounds__(kBlock) decode_down_kernel(
     const __nv_bfloat16* __restrict__ h, const __nv_bfloat16* __restrict__ wd, const int* __restrict__ cnt,
     const int* __restrict__ row_off, const int* __restrict__ touched, const int* __restrict__ hdr,
@@ -118,34 +163,28 @@ __global__ void __launch_bounds__(kBlock) decode_down_kernel(
     const int e = touched[u];
     const int c_e = cnt[e];
     const int r_e = row_off[e];
-    const __nv_bfloat16* w = wd + (static_cast<size_t>(e) * H + c0) * I;
+    const __nv_bfloat16* w[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) w[r] = wd + (static_cast<size_t>(e) * H + c0 + r) * I;
     for (int g0 = 0; g0 < c_e; g0 += 4) {
       const int ntok = min(4, c_e - g0);
-      const __nv_bfloat16* ht[4];
+      const __nv_bfloat16* a[4];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) ht[q] = h + static_cast<size_t>(r_e + g0 + min(q, ntok - 1)) * I;
-      float acc[32];
-#pragma unroll
-      for (int i = 0; i < 32; ++i) acc[i] = 0.f;
-      for (int ch = lane; ch < nch; ch += 32) {
-        uint4 a[8], hv[4];
-#pragma unroll
-        for (int rw = 0; rw < 8; ++rw) a[rw] = ld_stream_u4(w + static_cast<size_t>(rw) * I + ch * 8);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) hv[q] = *(reinterpret_cast<const uint4*>(ht[q]) + ch);
-#pragma unroll
-        for (int rw = 0; rw < 8; ++rw)
-#pragma unroll
-          for (int q = 0; q < 4; ++q) acc[rw * 4 + q] = dot8_bf16(a[rw], hv[q], acc[rw * 4 + q]);
+      for (int q = 0; q < 4; ++q) a[q] = h + static_cast<size_t>(r_e + g0 + min(q, ntok - 1)) * I;
+      const size_t row0 = static_cast<size_t>(r_e + g0);
+      switch (ntok) {
+        case 1: down_group<1>(w, a, nch, lane, y, row0, H, c0); break;
+        case 2: down_group<2>(w, a, nch, lane, y, row0, H, c0); break;
+        case 3: down_group<3>(w, a, nch, lane, y, row0, H, c0); break;
+        default: down_group<4>(w, a, nch, lane, y, row0, H, c0); break;
       }
-      const float sum = warp_transpose_reduce(acc, lane);
-      const int rw = lane >> 2, q = lane & 3;
-      if (q < ntok) y[static_cast<size_t>(r_e + g0 + q) * H + c0 + rw] = __float2bfloat16_rn(sum);
     }
   }
 }
 
 }  // namespace
+
+bool decode_supported(const moe_shape*) { return true; }
 
 // which = 0: gate/up (x -> h); which = 1: down (h -> y).
 cudaError_t launch_decode(const moe_shape* s, const Plan& p, const void* x, const void* w_gate_up,
@@ -157,8 +196,14 @@ cudaError_t launch_decode(const moe_shape* s, const Plan& p, const void* x, cons
   const int* hdr = reinterpret_cast<const int*>(ws + p.hdr);
   __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(ws + p.h);
   __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(ws + p.y);
-  // enough resident warps to keep ~100 KB of weight loads in flight per SM
-  const int grid = num_sms * 4;
+  // exactly one wave of resident blocks: every warp starts at once and the
+  // grid-stride task loop spreads the rows evenly over all of them
+  int per_sm = 0;
+  cudaError_t err = which == 0
+                        ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_gate_up_kernel, kBlock, 0)
+                        : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_down_kernel, kBlock, 0);
+  if (err != cudaSuccess) return err;
+  const int grid = num_sms * (per_sm < 1 ? 1 : per_sm);
   if (which == 0) {
     decode_gate_up_kernel<<<grid, kBlock, 0, st>>>(static_cast<const __nv_bfloat16*>(x),
                                                    static_cast<const __nv_bfloat16*>(w_gate_up), cnt, row_off,

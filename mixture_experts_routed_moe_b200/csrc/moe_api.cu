@@ -85,7 +85,8 @@ bool validate_shape(const moe_shape* s) {
 
 int resolve_path(const moe_shape* s) {
   if (s->path != MOE_PATH_AUTO) return s->path;
-  if (s->wdtype == MOE_DT_BF16 && static_cast<long long>(s->T) * s->k <= 4ll * s->E) return MOE_PATH_DECODE;
+  if (s->wdtype == MOE_DT_BF16 && static_cast<long long>(s->T) * s->k <= 4ll * s->E && decode_supported(s))
+    return MOE_PATH_DECODE;
   return MOE_PATH_PREFILL;
 }
 
@@ -149,6 +150,7 @@ moe_status forward_impl(const moe_shape* shape, const void* x, const int32_t* to
   // e4m3 experts: PREFILL only, and the down tile spans two 128-column scale blocks
   if (fp8 && (plan.path == MOE_PATH_DECODE || !e4m3_path_available() || shape->H % 256 != 0))
     return MOE_ERR_UNSUPPORTED;
+  if (plan.path == MOE_PATH_DECODE && !decode_supported(shape)) return MOE_ERR_UNSUPPORTED;
   if (shape->T == 0) return MOE_OK;
   if (x == nullptr || topk_idx == nullptr || topk_w == nullptr || w_gate_up == nullptr || w_down == nullptr ||
       out == nullptr || workspace == nullptr)

@@ -48,6 +48,7 @@ cudaError_t launch_gemm_e4m3(const moe_shape* s, const Plan& p, const void* x, c
                              int which, int num_sms, cudaStream_t st);
 bool e4m3_path_available();
 
+bool decode_supported(const moe_shape* s);
 cudaError_t launch_decode(const moe_shape* s, const Plan& p, const void* x, const void* w_gate_up,
                           const void* w_down, uint8_t* ws, int which, int num_sms, cudaStream_t st);
 
