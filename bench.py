@@ -252,7 +252,8 @@ def run_reference(args, world, rank):
 
 def workload_config(wl, path):
     return {"workload": wl.name, "T": wl.T, "H": wl.H, "I": wl.I, "E": wl.E, "k": wl.k, "wdtype": wl.wdtype,
-            "path": path, "l2": "flushed between steps (256 MiB write)", "parallelism": "replicas"}
+            "path": path, "l2": "flushed between steps (256 MiB write)", "parallelism": "replicas",
+            "launch": "CUDA graph of moe_route + moe_forward" if path != "oracle" else "cpu"}
 
 
 def stage_roofline(wl, path, stage_ms, n_touched, peaks, peak_src):
@@ -311,8 +312,13 @@ def run_ours(args, world, rank, local):
     def new_events(n):
         return [torch.cuda.Event(enable_timing=True) for _ in range(n)]
 
+    # the timed step is the captured graph of moe_route + moe_forward
+    graph = moe.MoEGraph(layer, wl.T, dev)
+    graph.x.copy_(xd)
+    graph.logits.copy_(ld)
     for _ in range(args.warmup):
         flush.zero_()
+        graph.replay()
         layer(xd, ld, out=out)
     torch.cuda.synchronize()
     ws = layer._workspace(wl.T, dev)
@@ -322,7 +328,6 @@ def run_ours(args, world, rank, local):
 
     K = args.steps
     ev_s, ev_e = new_events(K), new_events(K)
-    st_ev = [new_events(5) for _ in range(K)]
     clocks = ClockSampler(dev.index)
     barrier(world)
     torch.cuda.synchronize()
@@ -330,35 +335,46 @@ def run_ours(args, world, rank, local):
     for i in range(K):
         flush.zero_()
         ev_s[i].record(stream)
-        layer(xd, ld, out=out, events=st_ev[i])
+        graph.replay()
         ev_e[i].record(stream)
     torch.cuda.synchronize()
     barrier(world)
     clk = clocks.stop()
     step_ms = [ev_s[i].elapsed_time(ev_e[i]) for i in range(K)]
     total_ms = max_over_ranks(sum(step_ms), world)
-    stage_ms = {j: sum(st_ev[i][j - 1].elapsed_time(st_ev[i][j]) for i in range(K)) / K for j in range(1, 5)}
-    route_ms = sum(ev_s[i].elapsed_time(st_ev[i][0]) for i in range(K)) / K
 
-    # end to end through the public API with host buffers
+    # stage breakdown (and the dominant kernel's duration): the same kernels
+    # launched eagerly through moe_forward_timed, on the same inputs
+    st_s, st_ev = new_events(K), [new_events(5) for _ in range(K)]
+    torch.cuda.synchronize()
+    for i in range(K):
+        flush.zero_()
+        st_s[i].record(stream)
+        layer(xd, ld, out=out, events=st_ev[i])
+    torch.cuda.synchronize()
+    stage_ms = {j: sum(st_ev[i][j - 1].elapsed_time(st_ev[i][j]) for i in range(K)) / K for j in range(1, 5)}
+    route_ms = sum(st_s[i].elapsed_time(st_ev[i][0]) for i in range(K)) / K
+    eager_ms = sum(st_s[i].elapsed_time(st_ev[i][4]) for i in range(K)) / K
+
+    # end to end through the public API with host buffers: H2D of x and logits
+    # into the graph's inputs, the graph, D2H of the output
     xh = x.pin_memory()
     lh = logits.pin_memory()
     oh = torch.empty((wl.T, wl.H), dtype=torch.bfloat16).pin_memory()
-    xd2, ld2 = torch.empty_like(xd), torch.empty_like(ld)
     e2e_s, e2e_e = new_events(K), new_events(K)
     barrier(world)
     torch.cuda.synchronize()
     for i in range(K):
         flush.zero_()
         e2e_s[i].record(stream)
-        xd2.copy_(xh, non_blocking=True)
-        ld2.copy_(lh, non_blocking=True)
-        layer(xd2, ld2, out=out)
-        oh.copy_(out, non_blocking=True)
+        res = graph(xh, lh)
+        oh.copy_(res, non_blocking=True)
         e2e_e[i].record(stream)
     torch.cuda.synchronize()
     barrier(world)
     e2e_ms = max_over_ranks(sum(e2e_s[i].elapsed_time(e2e_e[i]) for i in range(K)), world)
+    if not torch.equal(graph.out, out):
+        raise RuntimeError("graph replay and eager forward disagree")
 
     peaks, peak_src = load_peaks()
     per_step_launches = 1 + (1 if wl.T <= 256 else 3) + 2 + 1  # route, permute, gate/up, down, combine
@@ -371,7 +387,7 @@ def run_ours(args, world, rank, local):
         "config": workload_config(wl, path),
         "tflops": wl.flops() * K * world / (total_ms / 1e3) / 1e12,
         "stages_ms": {"route": route_ms, "permute": stage_ms[1], "gate_up": stage_ms[2], "down": stage_ms[3],
-                      "combine": stage_ms[4]},
+                      "combine": stage_ms[4], "eager_step": eager_ms},
         "touched_experts": n_touched,
         "roofline": None,
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s",

@@ -215,6 +215,41 @@ class MoELayer:
         return out
 
 
-__all__ = ["lib", "route", "forward", "forward_noalloc", "workspace_size", "workspace_layout", "alloc_workspace",
+class MoEGraph:
+    """One layer step (moe_route + moe_forward) captured once in a CUDA graph for
+    a fixed token count, on static device buffers ``x``, ``logits`` and ``out``.
+    ``replay()`` reruns the captured kernels with no host-side work per step;
+    ``__call__(x, logits)`` copies new inputs into the static buffers first.
+    The library's launches are capture-safe: no allocation, no host
+    synchronisation, and one-time set-up done by the eager warm-up call."""
+
+    def __init__(self, layer: "MoELayer", T: int, device=None):
+        device = torch.device(device or "cuda")
+        self.layer = layer
+        self.x = torch.zeros((T, layer.H), dtype=torch.bfloat16, device=device)
+        self.logits = torch.zeros((T, layer.E), dtype=torch.float32, device=device)
+        self.out = torch.empty((T, layer.H), dtype=torch.bfloat16, device=device)
+        side = torch.cuda.Stream(device=device)
+        side.wait_stream(torch.cuda.current_stream(device))
+        with torch.cuda.stream(side):  # eager warm-up: workspace, kernel set-up
+            layer(self.x, self.logits, out=self.out)
+        torch.cuda.current_stream(device).wait_stream(side)
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            layer(self.x, self.logits, out=self.out)
+
+    def replay(self) -> torch.Tensor:
+        self.graph.replay()
+        return self.out
+
+    def __call__(self, x=None, logits=None) -> torch.Tensor:
+        if x is not None:
+            self.x.copy_(x, non_blocking=True)
+        if logits is not None:
+            self.logits.copy_(logits, non_blocking=True)
+        return self.replay()
+
+
+__all__ = ["lib", "route", "forward", "forward_noalloc", "MoEGraph", "workspace_size", "workspace_layout", "alloc_workspace",
            "read_device_status", "make_shape", "MoELayer", "MoeError", "MoeShape", "EXPORTS", "STATUS",
            "status_string", "PATH", "WDTYPE"]

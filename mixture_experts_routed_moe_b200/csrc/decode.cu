@@ -198,12 +198,16 @@ cudaError_t launch_decode(const moe_shape* s, const Plan& p, const void* x, cons
   __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(ws + p.y);
   // exactly one wave of resident blocks: every warp starts at once and the
   // grid-stride task loop spreads the rows evenly over all of them
-  int per_sm = 0;
-  cudaError_t err = which == 0
-                        ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_gate_up_kernel, kBlock, 0)
-                        : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_down_kernel, kBlock, 0);
-  if (err != cudaSuccess) return err;
-  const int grid = num_sms * (per_sm < 1 ? 1 : per_sm);
+  static int per_sm[2] = {0, 0};  // resident blocks per SM (same on every B200)
+  if (per_sm[which] == 0) {
+    int n = 0;
+    cudaError_t err = which == 0
+                          ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_gate_up_kernel, kBlock, 0)
+                          : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_down_kernel, kBlock, 0);
+    if (err != cudaSuccess) return err;
+    per_sm[which] = n < 1 ? 1 : n;
+  }
+  const int grid = num_sms * per_sm[which];
   if (which == 0) {
     decode_gate_up_kernel<<<grid, kBlock, 0, st>>>(static_cast<const __nv_bfloat16*>(x),
                                                    static_cast<const __nv_bfloat16*>(w_gate_up), cnt, row_off,

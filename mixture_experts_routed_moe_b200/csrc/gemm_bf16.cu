@@ -257,8 +257,8 @@ template <int kN, bool kSwiGLU>
 cudaError_t launch_one(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmParams& gp, int grid,
                        cudaStream_t st) {
   const size_t smem = Layout<kN>::bytes(gp.E);
-  cudaError_t err = cudaFuncSetAttribute(grouped_gemm_bf16_kernel<kN, kSwiGLU>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  static unsigned long long done = 0;
+  cudaError_t err = ensure_max_smem(reinterpret_cast<const void*>(grouped_gemm_bf16_kernel<kN, kSwiGLU>), &done);
   if (err != cudaSuccess) return err;
   grouped_gemm_bf16_kernel<kN, kSwiGLU><<<grid, kThreads, smem, st>>>(tmA, tmB, gp);
   return cudaGetLastError();

@@ -303,8 +303,8 @@ template <bool kGateUp>
 cudaError_t launch_one(const CUtensorMap& tmA, const CUtensorMap& tmB, const Fp8Params& fp, int grid,
                        cudaStream_t st) {
   const size_t smem = smem_bytes(fp.E);
-  cudaError_t err = cudaFuncSetAttribute(grouped_gemm_e4m3_kernel<kGateUp>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  static unsigned long long done = 0;
+  cudaError_t err = ensure_max_smem(reinterpret_cast<const void*>(grouped_gemm_e4m3_kernel<kGateUp>), &done);
   if (err != cudaSuccess) return err;
   grouped_gemm_e4m3_kernel<kGateUp><<<grid, kThreads, smem, st>>>(tmA, tmB, fp);
   return cudaGetLastError();

@@ -68,6 +68,20 @@ int device_sm_count() {
   return n;
 }
 
+cudaError_t ensure_max_smem(const void* kernel, unsigned long long* done) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  const unsigned long long bit = (dev < 64) ? (1ull << dev) : 0ull;
+  if (bit != 0 && (__atomic_load_n(done, __ATOMIC_ACQUIRE) & bit)) return cudaSuccess;
+  int optin = 0;
+  err = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  if (err != cudaSuccess) return err;
+  err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+  if (err == cudaSuccess && bit != 0) __atomic_fetch_or(done, bit, __ATOMIC_ACQ_REL);
+  return err;
+}
+
 bool validate_shape(const moe_shape* s) {
   if (s == nullptr) return false;
   if (s->T < 0 || s->H < 128 || s->I < 128 || s->H % 128 != 0 || s->I % 128 != 0) return false;

@@ -61,4 +61,9 @@ bool encode_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, size_t el
 
 int device_sm_count();
 
+// Sets a kernel's dynamic shared-memory limit to the device maximum once per
+// device (a host call kept out of the per-launch path, so launches can be
+// captured in CUDA graphs). `done` is one bitmask per kernel, bit = device.
+cudaError_t ensure_max_smem(const void* kernel, unsigned long long* done);
+
 }  // namespace moe

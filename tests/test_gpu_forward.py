@@ -159,3 +159,19 @@ def test_full_size_bf16_sampled(name):
     # every output row is finite and non-trivial
     o = out.float()
     assert torch.isfinite(o).all() and (o.abs().amax(dim=1) > 0).all()
+
+
+@pytest.mark.parametrize("name", ["tiny", "decode"])
+def test_graph_replay_matches_eager(name):
+    """MoEGraph (route + forward captured in a CUDA graph) gives the eager
+    result on new inputs copied into its static buffers."""
+    wl = G.WORKLOADS[name]
+    W = G.make_weights(wl, 0, device="cuda")
+    layer = moe.MoELayer(W["w_gate_up"], W["w_down"], wl.k)
+    g = moe.MoEGraph(layer, wl.T)
+    for seed in (21, 22):
+        x, L = G.make_activations(wl, seed)
+        got = g(x.cuda(), L.cuda()).clone()
+        ref = layer(x.cuda(), L.cuda())
+        torch.cuda.synchronize()
+        assert torch.equal(got, ref)
