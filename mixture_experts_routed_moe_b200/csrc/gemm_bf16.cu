@@ -114,6 +114,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     if (lane == 0) {
       // ---------------- TMA producer ----------------
+      const uint64_t pol_a = l2_policy_evict_last();
       int stage = 0;
       uint32_t ph = 0;
       bool ok = true;
@@ -126,7 +127,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           mbar_arrive_expect_tx(&full[stage], L::kStage);
-          tma_load_2d(sA + stage * L::kA, &tmA, &full[stage], kb * kBK, c.row0);
+          // A rows are re-read by every N block of the expert: ask L2 to keep them
+          tma_load_2d_hint(sA + stage * L::kA, &tmA, &full[stage], kb * kBK, c.row0, pol_a);
           tma_load_2d(sB + stage * L::kB, &tmB, &full[stage], kb * kBK, brow);
           if (kN == 256)
             tma_load_2d(sB + stage * L::kB + 128 * kBK * 2, &tmB, &full[stage], kb * kBK, brow + p.b_second_offset);

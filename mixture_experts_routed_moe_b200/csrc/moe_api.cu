@@ -131,6 +131,7 @@ bool make_plan(const moe_shape* s, Plan* p) {
   p->block_counts = take(static_cast<size_t>(p->nblk) * E * 4);
   p->cnt = take(E * 4);
   p->mt_base = take((E + 1) * 4);
+  p->pt_base = take((E + 1) * 4);
   p->touched = take(E * 4);
   p->local_rank = take(std::max<long long>(A, 1) * 4);
   p->row_src = take(std::max<size_t>(M, 1) * 4);
@@ -191,9 +192,13 @@ moe_status forward_impl(const moe_shape* shape, const void* x, const int32_t* to
     if (err != cudaSuccess || !mark(2)) return MOE_ERR_CUDA;
     err = launch_decode(shape, plan, x, w_gate_up, w_down, ws, 1, sms, st);
   } else if (!fp8) {
+    // gate/up: single-CTA 128x256 tiles; down: CTA-pair 256x256 tiles when
+    // H allows (each measured the faster of the two on the prefill-shaped and
+    // skewed layers)
     err = launch_gemm_bf16(shape, plan, w_gate_up, w_down, ws, 0, sms, st);
     if (err != cudaSuccess || !mark(2)) return MOE_ERR_CUDA;
-    err = launch_gemm_bf16(shape, plan, w_gate_up, w_down, ws, 1, sms, st);
+    err = shape->H % 256 == 0 ? launch_gemm_bf16_pair(shape, plan, w_gate_up, w_down, ws, 1, sms, st)
+                              : launch_gemm_bf16(shape, plan, w_gate_up, w_down, ws, 1, sms, st);
   } else {
     err = launch_gemm_e4m3(shape, plan, x, w_gate_up, w_down, sw_gate_up, sw_down, ws, 0, sms, st);
     if (err != cudaSuccess || !mark(2)) return MOE_ERR_CUDA;

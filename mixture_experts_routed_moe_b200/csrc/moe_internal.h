@@ -22,12 +22,12 @@ struct Plan {
   int bm;          // rows per expert tile: kTileM (PREFILL) or 1 (DECODE)
   int64_t m_rows;  // row capacity of the permuted buffers
   int nblk;        // permute blocks of kPermuteTokens tokens
-  size_t status, hdr, block_counts, cnt, mt_base, touched, local_rank, row_src, slot_row;
+  size_t status, hdr, block_counts, cnt, mt_base, pt_base, touched, local_rank, row_src, slot_row;
   size_t xa, xs, h, hs, y, total;
 };
 
 // Header words written on the device by the permute stage.
-enum HdrWord { kHdrMTiles = 0, kHdrTouched = 1, kHdrRows = 2 };
+enum HdrWord { kHdrMTiles = 0, kHdrTouched = 1, kHdrRows = 2, kHdrPairs = 3 };
 
 bool validate_shape(const moe_shape* s);
 int resolve_path(const moe_shape* s);
@@ -41,6 +41,10 @@ cudaError_t launch_permute(const moe_shape* s, const Plan& p, const int* topk_id
 
 cudaError_t launch_gemm_bf16(const moe_shape* s, const Plan& p, const void* w_gate_up, const void* w_down,
                              uint8_t* ws, int which, int num_sms, cudaStream_t st);
+
+// 2-CTA (cta_group::2) down projection (which = 1), for H % 256 == 0.
+cudaError_t launch_gemm_bf16_pair(const moe_shape* s, const Plan& p, const void* w_gate_up, const void* w_down,
+                                  uint8_t* ws, int which, int num_sms, cudaStream_t st);
 
 // which = 0 also quantises the permuted activations (x -> e4m3 codes + fp32 scales).
 cudaError_t launch_gemm_e4m3(const moe_shape* s, const Plan& p, const void* x, const void* w_gate_up,

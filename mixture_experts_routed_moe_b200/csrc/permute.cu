@@ -102,8 +102,9 @@ __device__ __forceinline__ int block_inclusive_scan(int v, int* s_warp) {
 // experts that received tokens. `counts` holds per-block counts on entry and
 // per-block exclusive bases on exit. Runs as one block of 1024 threads.
 __device__ __forceinline__ void scan_experts(int* __restrict__ counts, int nblk, int E, int bm, int* __restrict__ cnt,
-                                             int* __restrict__ mt_base, int* __restrict__ touched,
-                                             int* __restrict__ hdr, int* __restrict__ row_src, int* s_warp) {
+                                             int* __restrict__ mt_base, int* __restrict__ pt_base,
+                                             int* __restrict__ touched, int* __restrict__ hdr,
+                                             int* __restrict__ row_src, int* s_warp) {
   const int e = threadIdx.x;
   int c = 0;
   if (e < E) {
@@ -116,26 +117,32 @@ __device__ __forceinline__ void scan_experts(int* __restrict__ counts, int nblk,
   }
   const int tiles = (e < E) ? (c + bm - 1) / bm : 0;
   const int used = (e < E && c > 0) ? 1 : 0;
+  const int pairs = (tiles + 1) / 2;  // 256-row tile pairs of the 2-CTA GEMM
   const int tiles_incl = block_inclusive_scan(tiles, s_warp);
   const int used_incl = block_inclusive_scan(used, s_warp);
+  const int pairs_incl = block_inclusive_scan(pairs, s_warp);
   if (e < E) {
     const int base = tiles_incl - tiles;
     mt_base[e] = base;
+    pt_base[e] = pairs_incl - pairs;
     if (used) touched[used_incl - 1] = e;
     for (int r = base * bm + c; r < (base + tiles) * bm; ++r) row_src[r] = -1;
     if (e == E - 1) {
       mt_base[E] = tiles_incl;
+      pt_base[E] = pairs_incl;
       hdr[kHdrMTiles] = tiles_incl;
       hdr[kHdrTouched] = used_incl;
       hdr[kHdrRows] = tiles_incl * bm;
+      hdr[kHdrPairs] = pairs_incl;
     }
   }
 }
 
 __global__ void __launch_bounds__(1024) permute_scan_kernel(int* counts, int nblk, int E, int bm, int* cnt,
-                                                            int* mt_base, int* touched, int* hdr, int* row_src) {
+                                                            int* mt_base, int* pt_base, int* touched, int* hdr,
+                                                            int* row_src) {
   __shared__ int s_warp[32];
-  scan_experts(counts, nblk, E, bm, cnt, mt_base, touched, hdr, row_src, s_warp);
+  scan_experts(counts, nblk, E, bm, cnt, mt_base, pt_base, touched, hdr, row_src, s_warp);
 }
 
 // Copy one assignment's bf16 hidden-state row into its permuted row (one warp).
@@ -213,6 +220,7 @@ __global__ void __launch_bounds__(256) permute_scatter_kernel(const int* __restr
 // Everything in one block of 1024 threads, for T <= kPermuteTokens.
 __global__ void __launch_bounds__(1024) permute_small_kernel(const int* __restrict__ idx, int T, int k, int E, int bm,
                                                              int* __restrict__ cnt, int* __restrict__ mt_base,
+                                                             int* __restrict__ pt_base,
                                                              int* __restrict__ touched, int* __restrict__ hdr,
                                                              int* __restrict__ row_src, int* __restrict__ slot_row,
                                                              int* __restrict__ local_rank, int* dev_status,
@@ -244,20 +252,25 @@ __global__ void __launch_bounds__(1024) permute_small_kernel(const int* __restri
   const int e = threadIdx.x;
   const int tiles = (e < E) ? (c + bm - 1) / bm : 0;
   const int used = (e < E && c > 0) ? 1 : 0;
+  const int pairs = (tiles + 1) / 2;
   const int tiles_incl = block_inclusive_scan(tiles, s_warp);
   const int used_incl = block_inclusive_scan(used, s_warp);
+  const int pairs_incl = block_inclusive_scan(pairs, s_warp);
   if (e < E) {
     const int base = tiles_incl - tiles;
     cnt[e] = c;
     mt_base[e] = base;
+    pt_base[e] = pairs_incl - pairs;
     s_base[e] = base * bm;
     if (used) touched[used_incl - 1] = e;
     for (int r = base * bm + c; r < (base + tiles) * bm; ++r) row_src[r] = -1;
     if (e == E - 1) {
       mt_base[E] = tiles_incl;
+      pt_base[E] = pairs_incl;
       hdr[kHdrMTiles] = tiles_incl;
       hdr[kHdrTouched] = used_incl;
       hdr[kHdrRows] = tiles_incl * bm;
+      hdr[kHdrPairs] = pairs_incl;
     }
   }
   __syncthreads();
@@ -288,6 +301,7 @@ cudaError_t launch_permute(const moe_shape* s, const Plan& p, const int* topk_id
   int* counts = reinterpret_cast<int*>(ws + p.block_counts);
   int* cnt = reinterpret_cast<int*>(ws + p.cnt);
   int* mt_base = reinterpret_cast<int*>(ws + p.mt_base);
+  int* pt_base = reinterpret_cast<int*>(ws + p.pt_base);
   int* touched = reinterpret_cast<int*>(ws + p.touched);
   int* lrank = reinterpret_cast<int*>(ws + p.local_rank);
   int* row_src = reinterpret_cast<int*>(ws + p.row_src);
@@ -305,13 +319,14 @@ cudaError_t launch_permute(const moe_shape* s, const Plan& p, const int* topk_id
   cudaError_t err = cudaMemsetAsync(status, 0, sizeof(int), st);
   if (err != cudaSuccess) return err;
   if (T <= kSmallPermuteT) {
-    permute_small_kernel<<<1, 1024, mask_bytes, st>>>(topk_idx, T, k, E, p.bm, cnt, mt_base, touched, hdr, row_src,
+    permute_small_kernel<<<1, 1024, mask_bytes, st>>>(topk_idx, T, k, E, p.bm, cnt, mt_base, pt_base, touched, hdr,
+                                                      row_src,
                                                       slot_row, lrank, status, xb, xa, xq, xs, H);
     return cudaGetLastError();
   }
   permute_count_kernel<<<p.nblk, kPermuteTokens, mask_bytes, st>>>(topk_idx, T, k, E, counts, lrank, status);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
-  permute_scan_kernel<<<1, 1024, 0, st>>>(counts, p.nblk, E, p.bm, cnt, mt_base, touched, hdr, row_src);
+  permute_scan_kernel<<<1, 1024, 0, st>>>(counts, p.nblk, E, p.bm, cnt, mt_base, pt_base, touched, hdr, row_src);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   const long long A = static_cast<long long>(T) * k;
   permute_scatter_kernel<<<static_cast<unsigned>((A + 7) / 8), 256, 0, st>>>(
