@@ -282,8 +282,12 @@ def stage_roofline(wl, path, stage_ms, n_touched, peaks, peak_src):
             kern, src = ("gemm_e4m3_gate_up" if s == 1 else "gemm_e4m3_down"), "gemm_e4m3.cu"
         else:
             peak, how = peaks["bf16_tflops"], "measured bf16 burst"
-            kern, src = ("grouped_gemm_bf16_kernel<256,true>" if s == 1 else "grouped_gemm_bf16_kernel<256,false>"), \
-                "gemm_bf16.cu"
+            # gate/up: single-CTA kernel; down: the CTA-pair kernel when H % 256 == 0
+            if s == 1:
+                kern, src = "grouped_gemm_bf16_kernel<256,true>", "gemm_bf16.cu"
+            else:
+                kern, src = (("grouped_gemm_bf16_pair_kernel", "gemm_bf16_pair.cu") if H % 256 == 0
+                             else ("grouped_gemm_bf16_kernel<128,false>", "gemm_bf16.cu"))
         out = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
                "kernel": kern, "stage": names[s], "algorithmic_flops": flops, "peak_source": how}
     rec = NCU_TRAFFIC.get((wl.name, kern))
