@@ -418,7 +418,13 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=list(G.WORKLOADS), default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--shape", default=None,
+                    help="T,H,I,E,k,wdtype: a custom layer instead of a named workload (profiling-sized cases)")
     args = ap.parse_args()
+    if args.shape:
+        T, H, I, E, k, wd = args.shape.split(",")
+        G.WORKLOADS["custom"] = G.Workload("custom", int(T), int(H), int(I), int(E), int(k), wdtype=wd)
+        args.workload = "custom"
     if args.warmup < 3 and args.impl == "ours":
         log("note: fewer than 3 warm-up steps")
     if args.impl == "reference":

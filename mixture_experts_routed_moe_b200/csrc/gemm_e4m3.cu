@@ -122,6 +122,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     if (lane == 0) {
       // ---------------- TMA producer ----------------
+      // weights stream through L2 once; the activation tile is re-read by
+      // every column block of the expert: keep it, drop the weights first
+      const uint64_t pol_a = l2_policy_evict_last();
+      const uint64_t pol_b = l2_policy_evict_first();
       int stage = 0;
       uint32_t ph = 0;
       bool ok = true;
@@ -134,9 +138,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           mbar_arrive_expect_tx(&full[stage], kStage);
-          tma_load_2d(sA + stage * kA, &tmA, &full[stage], kb * kBK, c.row0);
-          tma_load_2d(sB + stage * kB, &tmB, &full[stage], kb * kBK, brow);
-          tma_load_2d(sB + stage * kB + 128 * kBK, &tmB, &full[stage], kb * kBK, brow + p.b_second_offset);
+          tma_load_2d_hint(sA + stage * kA, &tmA, &full[stage], kb * kBK, c.row0, pol_a);
+          tma_load_2d_hint(sB + stage * kB, &tmB, &full[stage], kb * kBK, brow, pol_b);
+          tma_load_2d_hint(sB + stage * kB + 128 * kBK, &tmB, &full[stage], kb * kBK, brow + p.b_second_offset, pol_b);
           if (++stage == kStages) {
             stage = 0;
             ph ^= 1;
