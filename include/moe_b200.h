@@ -57,6 +57,14 @@ typedef enum {
   MOE_PATH_DECODE = 2   /* weight-streaming kernels, no tile padding (bf16 only) */
 } moe_path;
 
+/* Gate activation of the gated expert MLP (section "SonicMoE": SwiGLU, GeGLU
+ * and ReGLU map to silu, gelu and relu). h = act(gate) * up. */
+typedef enum {
+  MOE_ACT_SILU = 0, /* SwiGLU: silu(g) = g / (1 + exp(-g)) */
+  MOE_ACT_GELU = 1, /* GeGLU:  gelu(g) = g/2 * (1 + erf(g / sqrt 2)), the exact form */
+  MOE_ACT_RELU = 2  /* ReGLU:  relu(g) = max(g, 0) */
+} moe_activation;
+
 /* Problem shape. T tokens, hidden size H, expert intermediate size I,
  * E experts, top-k. Requirements: T >= 0; H and I positive multiples of 128;
  * 1 <= E <= 1024; 1 <= k <= E; T*k < 2^31 and every buffer below 2^31 rows. */
@@ -64,6 +72,7 @@ typedef struct {
   int32_t T, H, I, E, k;
   int32_t wdtype; /* moe_wdtype */
   int32_t path;   /* moe_path */
+  int32_t act;    /* moe_activation */
 } moe_shape;
 
 /*
@@ -88,7 +97,8 @@ size_t moe_workspace_size(const moe_shape* shape);
 /*
  * moe_forward -- the routed expert forward ("Experts backends", introduction;
  * the "eager" row of the backend table is its reference definition):
- *   out[t] = sum_j topk_w[t,j] * Wd[e] (silu(Wg[e] x[t]) * (Wu[e] x[t])),  e = topk_idx[t,j]
+ *   out[t] = sum_j topk_w[t,j] * Wd[e] (act(Wg[e] x[t]) * (Wu[e] x[t])),  e = topk_idx[t,j]
+ * with act = shape->act (silu for SwiGLU experts).
  *
  *   x          [T, H] bf16
  *   topk_idx   [T, k] int32, each row k distinct experts in [0, E)
@@ -102,7 +112,7 @@ size_t moe_workspace_size(const moe_shape* shape);
  *   workspace  >= moe_workspace_size(shape) bytes, 256-byte aligned; its
  *              previous contents do not matter. Calls that share a workspace
  *              must not overlap in time.
- * Intermediates: h = silu(gate) * up is rounded to bf16 and the expert output
+ * Intermediates: h = act(gate) * up is rounded to bf16 and the expert output
  * y to bf16 (e4m3 experts: x and h are quantised per token and per 128-column
  * group with an fp32 scale amax/448, the FP8 reading of section "FP8 and FP4
  * quantized experts"; y stays bf16). The weighted sum runs in fp32 over j in

@@ -25,6 +25,7 @@ STATUS = {
 }
 WDTYPE = {"bf16": 0, "e4m3": 1}
 PATH = {"auto": 0, "prefill": 1, "decode": 2}
+ACT = {"silu": 0, "gelu": 1, "relu": 2}
 PATH_NAMES = {v: k for k, v in PATH.items()}
 EXPORTS = ["moe_route", "moe_workspace_size", "moe_forward", "moe_forward_timed", "moe_workspace_query",
            "moe_read_device_status", "moe_status_string", "moe_version", "moe_forward_noalloc"]
@@ -38,7 +39,7 @@ class MoeError(RuntimeError):
 
 class MoeShape(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int32), ("H", ctypes.c_int32), ("I", ctypes.c_int32), ("E", ctypes.c_int32),
-                ("k", ctypes.c_int32), ("wdtype", ctypes.c_int32), ("path", ctypes.c_int32)]
+                ("k", ctypes.c_int32), ("wdtype", ctypes.c_int32), ("path", ctypes.c_int32), ("act", ctypes.c_int32)]
 
 
 class MoeWorkspaceLayout(ctypes.Structure):
@@ -100,9 +101,9 @@ def _stream(stream=None):
     return ctypes.c_void_p(s.cuda_stream)
 
 
-def make_shape(T, H, I, E, k, wdtype="bf16", path="auto") -> MoeShape:
+def make_shape(T, H, I, E, k, wdtype="bf16", path="auto", act="silu") -> MoeShape:
     return MoeShape(int(T), int(H), int(I), int(E), int(k), WDTYPE[wdtype] if isinstance(wdtype, str) else int(wdtype),
-                    PATH[path] if isinstance(path, str) else int(path))
+                    PATH[path] if isinstance(path, str) else int(path), ACT[act] if isinstance(act, str) else int(act))
 
 
 def workspace_size(shape: MoeShape) -> int:
@@ -137,15 +138,16 @@ def route(logits: torch.Tensor, k: int, topk_idx: torch.Tensor | None = None, to
 
 
 def forward(x, topk_idx, topk_w, w_gate_up, w_down, sw_gate_up=None, sw_down=None, out=None, workspace=None,
-            path="auto", stream=None, events=None):
+            path="auto", stream=None, events=None, act="silu"):
     """moe_forward: bf16 x [T,H] with routing [T,k] through experts
     w_gate_up [E,2I,H], w_down [E,H,I] (bf16, or float8_e4m3fn with uint8 UE8M0
-    block scales) -> bf16 out [T,H]. Returns (out, workspace)."""
+    block scales) -> bf16 out [T,H]; act is the gate activation ("silu" for
+    SwiGLU, "gelu" for GeGLU, "relu" for ReGLU). Returns (out, workspace)."""
     T, H = x.shape
     k = topk_idx.shape[1]
     E, twoI, _ = w_gate_up.shape
     wdtype = "e4m3" if w_gate_up.dtype == torch.float8_e4m3fn else "bf16"
-    shape = make_shape(T, H, twoI // 2, E, k, wdtype, path)
+    shape = make_shape(T, H, twoI // 2, E, k, wdtype, path, act)
     if out is None:
         out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device)
     if workspace is None:
@@ -164,7 +166,7 @@ def forward(x, topk_idx, topk_w, w_gate_up, w_down, sw_gate_up=None, sw_down=Non
 
 
 def forward_noalloc(x, topk_idx, topk_w, w_gate_up, w_down, sw_gate_up=None, sw_down=None, out=None, path="auto",
-                    stream=None):
+                    stream=None, act="silu"):
     """moe_forward_noalloc: the forward with the library's own fixed scratch
     array instead of a caller workspace, for callers that cannot allocate device
     memory (only ``out`` is allocated here when not given). Calls share the
@@ -173,7 +175,7 @@ def forward_noalloc(x, topk_idx, topk_w, w_gate_up, w_down, sw_gate_up=None, sw_
     k = topk_idx.shape[1]
     E, twoI, _ = w_gate_up.shape
     wdtype = "e4m3" if w_gate_up.dtype == torch.float8_e4m3fn else "bf16"
-    shape = make_shape(T, H, twoI // 2, E, k, wdtype, path)
+    shape = make_shape(T, H, twoI // 2, E, k, wdtype, path, act)
     if out is None:
         out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device)
     _check(lib().moe_forward_noalloc(ctypes.byref(shape), _ptr(x), _ptr(topk_idx), _ptr(topk_w), _ptr(w_gate_up),
@@ -192,17 +194,17 @@ class MoELayer:
     runs moe_route then moe_forward and returns bf16 [T,H]. The workspace is
     allocated once per shape and reused."""
 
-    def __init__(self, w_gate_up, w_down, k, sw_gate_up=None, sw_down=None, path="auto"):
+    def __init__(self, w_gate_up, w_down, k, sw_gate_up=None, sw_down=None, path="auto", act="silu"):
         self.w_gate_up, self.w_down = w_gate_up, w_down
         self.sw_gate_up, self.sw_down = sw_gate_up, sw_down
-        self.k, self.path = int(k), path
+        self.k, self.path, self.act = int(k), path, act
         self.E, twoI, self.H = w_gate_up.shape
         self.I = twoI // 2
         self._ws = {}
 
     def _workspace(self, T, device):
         wdtype = "e4m3" if self.w_gate_up.dtype == torch.float8_e4m3fn else "bf16"
-        shape = make_shape(T, self.H, self.I, self.E, self.k, wdtype, self.path)
+        shape = make_shape(T, self.H, self.I, self.E, self.k, wdtype, self.path, self.act)
         key = (T, str(device))
         if key not in self._ws:
             self._ws[key] = alloc_workspace(shape, device)
@@ -211,7 +213,8 @@ class MoELayer:
     def __call__(self, x, logits, out=None, events=None):
         idx, w = route(logits, self.k)
         out, _ = forward(x, idx, w, self.w_gate_up, self.w_down, self.sw_gate_up, self.sw_down, out=out,
-                         workspace=self._workspace(x.shape[0], x.device), path=self.path, events=events)
+                         workspace=self._workspace(x.shape[0], x.device), path=self.path, events=events,
+                         act=self.act)
         return out
 
 
@@ -252,4 +255,4 @@ class MoEGraph:
 
 __all__ = ["lib", "route", "forward", "forward_noalloc", "MoEGraph", "workspace_size", "workspace_layout", "alloc_workspace",
            "read_device_status", "make_shape", "MoELayer", "MoeError", "MoeShape", "EXPORTS", "STATUS",
-           "status_string", "PATH", "WDTYPE"]
+           "status_string", "PATH", "WDTYPE", "ACT"]

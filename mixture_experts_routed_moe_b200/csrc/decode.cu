@@ -11,7 +11,7 @@
 // cores: the work is bound by HBM. The grid is exactly one wave of resident
 // blocks.
 //
-//   gate/up:  h[row, n] = silu(<x_t, Wg_e[n]>) * <x_t, Wu_e[n]>  (bf16)
+//   gate/up:  h[row, n] = act(<x_t, Wg_e[n]>) * <x_t, Wu_e[n]>   (bf16)
 //   down:     y[row, c] = <h[row], Wd_e[c]>                      (bf16)
 //
 // Rows are the unpadded expert-major permuted rows (tile size 1).
@@ -71,7 +71,8 @@ __device__ __forceinline__ void dot_rows(const __nv_bfloat16* const (&w)[NR], co
 // weight rows 0..3 are gate rows n0.., rows 4..7 the up rows I+n0...
 template <int NQ>
 __device__ __forceinline__ void gate_up_group(const __nv_bfloat16* const (&w)[8], const __nv_bfloat16* const (&a)[4],
-                                              int nch, int lane, __nv_bfloat16* h, size_t row0, int I, int n0) {
+                                              int nch, int lane, __nv_bfloat16* h, size_t row0, int I, int n0,
+                                              int act) {
   float acc[8][4];
 #pragma unroll
   for (int r = 0; r < 8; ++r)
@@ -83,14 +84,14 @@ __device__ __forceinline__ void gate_up_group(const __nv_bfloat16* const (&w)[8]
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
       const float g = warp_sum(acc[r][q]), u = warp_sum(acc[4 + r][q]);
-      if (lane == r) h[(row0 + q) * I + n0 + r] = __float2bfloat16_rn(swiglu(g, u));
+      if (lane == r) h[(row0 + q) * I + n0 + r] = __float2bfloat16_rn(gated_act(act, g, u));
     }
 }
 
 __global__ void __launch_bounds__(kBlock) decode_gate_up_kernel(
     const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ wgu, const int* __restrict__ cnt,
     const int* __restrict__ row_off, const int* __restrict__ row_src, const int* __restrict__ touched,
-    const int* __restrict__ hdr, __nv_bfloat16* __restrict__ h, int H, int I, int k) {
+    const int* __restrict__ hdr, __nv_bfloat16* __restrict__ h, int H, int I, int k, int act) {
   const int lane = threadIdx.x & 31;
   const int gwarp = blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
   const int nwarps = gridDim.x * kWarpsPerBlock;
@@ -118,10 +119,10 @@ __global__ void __launch_bounds__(kBlock) decode_gate_up_kernel(
       for (int q = 0; q < 4; ++q) a[q] = x + static_cast<size_t>(row_src[r_e + g0 + min(q, ntok - 1)] / k) * H;
       const size_t row0 = static_cast<size_t>(r_e + g0);
       switch (ntok) {
-        case 1: gate_up_group<1>(w, a, nch, lane, h, row0, I, n0); break;
-        case 2: gate_up_group<2>(w, a, nch, lane, h, row0, I, n0); break;
-        case 3: gate_up_group<3>(w, a, nch, lane, h, row0, I, n0); break;
-        default: gate_up_group<4>(w, a, nch, lane, h, row0, I, n0); break;
+        case 1: gate_up_group<1>(w, a, nch, lane, h, row0, I, n0, act); break;
+        case 2: gate_up_group<2>(w, a, nch, lane, h, row0, I, n0, act); break;
+        case 3: gate_up_group<3>(w, a, nch, lane, h, row0, I, n0, act); break;
+        default: gate_up_group<4>(w, a, nch, lane, h, row0, I, n0, act); break;
       }
     }
   }
@@ -211,7 +212,7 @@ cudaError_t launch_decode(const moe_shape* s, const Plan& p, const void* x, cons
   if (which == 0) {
     decode_gate_up_kernel<<<grid, kBlock, 0, st>>>(static_cast<const __nv_bfloat16*>(x),
                                                    static_cast<const __nv_bfloat16*>(w_gate_up), cnt, row_off,
-                                                   row_src, touched, hdr, h, s->H, s->I, s->k);
+                                                   row_src, touched, hdr, h, s->H, s->I, s->k, s->act);
   } else {
     decode_down_kernel<<<grid, kBlock, 0, st>>>(h, static_cast<const __nv_bfloat16*>(w_down), cnt, row_off, touched,
                                                 hdr, y, s->H, s->I);

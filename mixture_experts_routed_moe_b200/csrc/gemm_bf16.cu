@@ -4,7 +4,7 @@
 // down projection; grouped_mm / deepgemm run all experts in one grouped GEMM
 // over expert-sorted tokens):
 //
-//   gate/up:  h[rows of e, n..n+127] = silu(X_e Wg_e^T) * (X_e Wu_e^T)   (SwiGLU in the epilogue)
+//   gate/up:  h[rows of e, n..n+127] = act(X_e Wg_e^T) * (X_e Wu_e^T)   (SwiGLU/GeGLU/ReGLU in the epilogue)
 //   down:     y[rows of e, n..n+N-1] = h_e Wd_e^T
 //
 // Tile = (expert e, 128-row block of e's permuted rows, N-column block). The
@@ -45,6 +45,7 @@ struct GemmParams {
   __nv_bfloat16* out;
   int out_ld;         // elements per output row
   int out_tile_cols;  // output columns per tile
+  int act;  // gate activation (moe_activation)
   int* dev_status;
   unsigned long long timeout_ns;
 };
@@ -216,8 +217,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i)
-            pk[i] = pack_bf16x2(swiglu(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i])),
-                                swiglu(__uint_as_float(g[2 * i + 1]), __uint_as_float(u[2 * i + 1])));
+            pk[i] = pack_bf16x2(gated_act(p.act, __uint_as_float(g[2 * i]), __uint_as_float(u[2 * i])),
+                                gated_act(p.act, __uint_as_float(g[2 * i + 1]), __uint_as_float(u[2 * i + 1])));
           if (valid) {
             uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
 #pragma unroll
@@ -278,6 +279,7 @@ cudaError_t launch_gemm_bf16(const moe_shape* s, const Plan& p, const void* w_ga
   gp.E = E;
   gp.dev_status = reinterpret_cast<int*>(ws + p.status);
   gp.timeout_ns = kDefaultTimeoutNs;
+  gp.act = s->act;
   // every tile count is bounded by the row capacity
   const int max_mtiles = static_cast<int>(p.m_rows / kTileM);
   CUtensorMap tmA, tmB;

@@ -3,7 +3,7 @@
 // dynamic per-row activation scales; on Blackwell the expert weight scales are
 // UE8M0 powers of two, one per 128x128 block).
 //
-//   gate/up:  h = silu(Xg) * Xu with X = q_x * s_x (per row, per 128 columns) and
+//   gate/up:  h = act(Xg) * Xu with X = q_x * s_x (per row, per 128 columns) and
 //             W = q_w * 2^(b-127) (per 128x128 block); h is quantised again per
 //             row and 128 columns (e4m3 codes + fp32 scale)
 //   down:     y = h W_d^T, rounded to bf16
@@ -56,6 +56,7 @@ struct Fp8Params {
   float* hs;              // gate/up: h scales [m_rows, I/128]
   __nv_bfloat16* y;       // down: [m_rows, H]
   int out_ld;             // I (gate/up) or H (down)
+  int act;                // gate activation (moe_activation)
   int* dev_status;
   unsigned long long timeout_ns;
 };
@@ -260,7 +261,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float amax = 0.f;
 #pragma unroll
         for (int i = 0; i < 64; ++i) {
-          acc[i] = swiglu(acc[i], acc[64 + i]);
+          acc[i] = gated_act(p.act, acc[i], acc[64 + i]);
           amax = fmaxf(amax, fabsf(acc[i]));
         }
         s_amax[hf * kTileM + r] = amax;
@@ -330,6 +331,7 @@ cudaError_t launch_gemm_e4m3(const moe_shape* s, const Plan& p, const void* /*x*
   fp.E = E;
   fp.dev_status = reinterpret_cast<int*>(ws + p.status);
   fp.timeout_ns = kDefaultTimeoutNs;
+  fp.act = s->act;
   const int max_mtiles = static_cast<int>(p.m_rows / kTileM);
   CUtensorMap tmA, tmB;
   if (which == 0) {

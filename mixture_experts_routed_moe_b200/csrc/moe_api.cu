@@ -89,6 +89,7 @@ bool validate_shape(const moe_shape* s) {
   if (s->E < 1 || s->E > 1024 || s->k < 1 || s->k > s->E) return false;
   if (s->wdtype != MOE_DT_BF16 && s->wdtype != MOE_DT_E4M3) return false;
   if (s->path != MOE_PATH_AUTO && s->path != MOE_PATH_PREFILL && s->path != MOE_PATH_DECODE) return false;
+  if (s->act != MOE_ACT_SILU && s->act != MOE_ACT_GELU && s->act != MOE_ACT_RELU) return false;
   const long long A = static_cast<long long>(s->T) * s->k;
   const long long rows = A + static_cast<long long>(std::min<long long>(s->E, A)) * (kTileM - 1) + kTileM;
   if (rows >= (1ll << 31) || static_cast<long long>(s->E) * 2 * s->I >= (1ll << 31) ||

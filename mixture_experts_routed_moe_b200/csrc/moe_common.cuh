@@ -305,8 +305,19 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 
-// silu(g) * u in fp32: silu(z) = z / (1 + exp(-z)).
-__device__ __forceinline__ float swiglu(float g, float u) { return g / (1.0f + __expf(-g)) * u; }
+// act(g) * u in fp32 for the gated activations (moe_activation):
+// silu(z) = z / (1 + exp(-z)), gelu(z) = z/2 * (1 + erf(z / sqrt 2)), relu(z) = max(z, 0).
+// `act` is uniform across a kernel, so the branch never diverges.
+__device__ __forceinline__ float gated_act(int act, float g, float u) {
+  float a;
+  if (act == 1)
+    a = 0.5f * g * (1.0f + erff(g * 0.7071067811865476f));
+  else if (act == 2)
+    a = fmaxf(g, 0.0f);
+  else
+    a = g / (1.0f + __expf(-g));
+  return a * u;
+}
 
 // Streaming 16-byte load that does not allocate in L1.
 __device__ __forceinline__ uint4 ld_stream_u4(const void* p) {

@@ -16,7 +16,8 @@ implementation: a loop over the selected experts that applies the projections
 to their tokens. That eager loop is the algorithm written out here. The expert
 is a gated MLP: up projection, SwiGLU, down projection (backend table, row
 "deepgemm_megamoe"; section "Fused Mega MoE on Blackwell"), and the section
-"SonicMoE" maps the gated activations SwiGLU/GeGLU/ReGLU to silu/gelu/relu.
+"SonicMoE" maps the gated activations SwiGLU/GeGLU/ReGLU to silu/gelu/relu;
+all three are supported (gelu in its exact erf form).
 
 Arithmetic is float64 throughout. The pages fix no precision; where they are
 silent this module takes the readings below (each one is also listed in the
@@ -202,9 +203,27 @@ def silu(z):
         return z / (1.0 + np.exp(-z))
 
 
-def expert_mlp(X, w_gate_up_e, w_down_e, intermediate: str = "bf16"):
+def gelu(z):
+    """gelu(z) = z * Phi(z) = z/2 * (1 + erf(z / sqrt 2)), the exact (erf) form
+    (section "SonicMoE": gelu <-> GeGLU). erf from scipy."""
+    import scipy.special
+
+    z = np.asarray(z, dtype=np.float64)
+    return 0.5 * z * (1.0 + scipy.special.erf(z / np.sqrt(2.0)))
+
+
+def relu(z):
+    """relu(z) = max(z, 0) (section "SonicMoE": relu <-> ReGLU)."""
+    return np.maximum(np.asarray(z, dtype=np.float64), 0.0)
+
+
+ACTIVATIONS = {"silu": silu, "gelu": gelu, "relu": relu}
+
+
+def expert_mlp(X, w_gate_up_e, w_down_e, intermediate: str = "bf16", act: str = "silu"):
     """One expert's gated MLP on its tokens X [n, H] (float64):
-    up projection (gate and up halves of w_gate_up_e), SwiGLU, down projection.
+    up projection (gate and up halves of w_gate_up_e), gated activation
+    act(gate) * up (SwiGLU by default), down projection.
     Backend table, row "deepgemm_megamoe" (up projection, SwiGLU, down projection)."""
     I = w_gate_up_e.shape[0] // 2
     Wg = np.asarray(w_gate_up_e[:I], dtype=np.float64)
@@ -212,7 +231,7 @@ def expert_mlp(X, w_gate_up_e, w_down_e, intermediate: str = "bf16"):
     Wd = np.asarray(w_down_e, dtype=np.float64)
     G = X @ Wg.T
     U = X @ Wu.T
-    h = silu(G) * U
+    h = ACTIVATIONS[act](G) * U
     if intermediate == "bf16":
         h = bf16_round(h)
     y = h @ Wd.T
@@ -250,14 +269,15 @@ def combine(Y, topk_w, intermediate: str = "bf16"):
 
 
 def moe_forward(x, topk_idx, topk_w, w_gate_up, w_down, intermediate: str = "bf16",
-                tokens=None):
+                tokens=None, act: str = "silu"):
     """Routed MoE forward for bf16 experts.
 
     x [T,H]; topk_idx int [T,k]; topk_w fp32 [T,k]; w_gate_up [E,2I,H];
     w_down [E,H,I] (any float arrays holding the bf16 values). ``tokens``
     restricts the computation to a subset of tokens (each output row depends
     only on its own token). ``intermediate``: "bf16" (R4), "exact" (round the
-    output only) or "none" (no rounding at all). Returns float64 [len(tokens), H]."""
+    output only) or "none" (no rounding at all). ``act``: the gate activation
+    ("silu", "gelu" or "relu"). Returns float64 [len(tokens), H]."""
     x = np.asarray(x, dtype=np.float64)
     T = x.shape[0]
     tokens = np.arange(T) if tokens is None else np.asarray(tokens, dtype=np.int64)
@@ -265,7 +285,7 @@ def moe_forward(x, topk_idx, topk_w, w_gate_up, w_down, intermediate: str = "bf1
     mode = "bf16" if intermediate == "bf16" else "exact"
 
     def mlp(e, X):
-        return expert_mlp(X, w_gate_up[e], w_down[e], mode)[1]
+        return expert_mlp(X, w_gate_up[e], w_down[e], mode, act)[1]
 
     Y = _expert_loop(x, topk_idx, E, tokens, mlp)
     w = np.asarray(topk_w)[tokens]
@@ -307,7 +327,7 @@ def quantize_1x128(a):
     return codes, s, deq.reshape(R, C)
 
 
-def expert_mlp_fp8(X, wgu_codes, wgu_sb, wd_codes, wd_sb, quantize_acts: bool = True):
+def expert_mlp_fp8(X, wgu_codes, wgu_sb, wd_codes, wd_sb, quantize_acts: bool = True, act: str = "silu"):
     """One FP8 expert on its tokens X [n,H] (bf16 values): x quantised 1x128,
     gate/up projection, SwiGLU evaluated on the fp32 result, h quantised 1x128,
     down projection, y rounded to bf16."""
@@ -317,13 +337,13 @@ def expert_mlp_fp8(X, wgu_codes, wgu_sb, wd_codes, wd_sb, quantize_acts: bool = 
     Xq = quantize_1x128(X)[2] if quantize_acts else np.asarray(X, dtype=np.float64)
     G = Xq @ Wgu[:I].T
     U = Xq @ Wgu[I:].T
-    h = (silu(G) * U).astype(np.float32)
+    h = (ACTIVATIONS[act](G) * U).astype(np.float32)
     hq = quantize_1x128(h)[2] if quantize_acts else h.astype(np.float64)
     return bf16_round(hq @ Wd.T)
 
 
 def moe_forward_fp8(x, topk_idx, topk_w, wgu_codes, wgu_sb, wd_codes, wd_sb,
-                    tokens=None, quantize_acts: bool = True):
+                    tokens=None, quantize_acts: bool = True, act: str = "silu"):
     """Routed MoE forward for FP8 experts (e4m3 codes + UE8M0 block bytes).
     Shapes: wgu_codes uint8 [E,2I,H], wgu_sb uint8 [E,2I/128,H/128],
     wd_codes uint8 [E,H,I], wd_sb uint8 [E,H/128,I/128]. Returns float64 [len(tokens),H]."""
@@ -333,7 +353,7 @@ def moe_forward_fp8(x, topk_idx, topk_w, wgu_codes, wgu_sb, wd_codes, wd_sb,
     E = wgu_codes.shape[0]
 
     def mlp(e, X):
-        return expert_mlp_fp8(X, wgu_codes[e], wgu_sb[e], wd_codes[e], wd_sb[e], quantize_acts)
+        return expert_mlp_fp8(X, wgu_codes[e], wgu_sb[e], wd_codes[e], wd_sb[e], quantize_acts, act)
 
     Y = _expert_loop(x, topk_idx, E, tokens, mlp)
     return combine(Y, np.asarray(topk_w)[tokens], "bf16")

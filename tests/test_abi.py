@@ -49,7 +49,7 @@ def shape(**kw):
 
 
 @pytest.mark.parametrize("bad", [dict(H=100), dict(I=64), dict(E=0), dict(E=1025), dict(k=0), dict(k=9),
-                                 dict(T=-1), dict(wdtype=7), dict(path=9), dict(H=0)])
+                                 dict(T=-1), dict(wdtype=7), dict(path=9), dict(H=0), dict(act=3)])
 def test_invalid_shapes_rejected(L, bad):
     s = shape(**bad)
     assert L.moe_workspace_size(ctypes.byref(s)) == 0

@@ -175,3 +175,19 @@ def test_graph_replay_matches_eager(name):
         ref = layer(x.cuda(), L.cuda())
         torch.cuda.synchronize()
         assert torch.equal(got, ref)
+
+
+@pytest.mark.parametrize("act", ["gelu", "relu"])
+@pytest.mark.parametrize("path", ["prefill", "decode"])
+@pytest.mark.parametrize("name", ["tiny", "decode"])
+def test_gated_activations(name, path, act):
+    """GeGLU and ReGLU experts (section SonicMoE's silu/gelu/relu gates) on both paths."""
+    wl = G.WORKLOADS[name]
+    x, L, W = device_inputs(wl, 31)
+    idx, w, _ = O.route(L.numpy(), wl.k)
+    out, ws = moe.forward(x.cuda(), torch.from_numpy(idx).cuda(), torch.from_numpy(w).cuda(), W["w_gate_up"],
+                          W["w_down"], path=path, act=act)
+    torch.cuda.synchronize()
+    assert moe.read_device_status(ws) == 0
+    ref = O.moe_forward(x.float().numpy(), idx, w, ExpertView(W["w_gate_up"]), ExpertView(W["w_down"]), act=act)
+    assert_bf16_close(out.float().cpu().numpy(), ref, f"{name}/{path}/{act}")

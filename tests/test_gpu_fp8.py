@@ -98,3 +98,17 @@ def test_fp8_full_size_sampled():
     ref = oracle_forward_fp8(x, idx, w, W, tokens=toks)
     assert_fp8_close(out.float().cpu().numpy()[toks], ref, "fp8 full")
     assert torch.isfinite(out.float()).all()
+
+
+@pytest.mark.parametrize("act", ["gelu", "relu"])
+def test_fp8_gated_activations(act):
+    wl = G.Workload("fp8act", 64, 256, 256, 8, 2, wdtype="e4m3")
+    x, L, W = device_inputs(wl, 6)
+    idx, w, _ = O.route(L.numpy(), wl.k)
+    out, ws = moe.forward(x.cuda(), torch.from_numpy(idx).cuda(), torch.from_numpy(w).cuda(), W["w_gate_up"],
+                          W["w_down"], W["sw_gate_up"], W["sw_down"], act=act)
+    torch.cuda.synchronize()
+    ref = O.moe_forward_fp8(x.float().numpy(), idx, w, ExpertView(W["w_gate_up"], True),
+                            ExpertView(W["sw_gate_up"], True), ExpertView(W["w_down"], True),
+                            ExpertView(W["sw_down"], True), act=act)
+    assert assert_fp8_close(out.float().cpu().numpy(), ref, f"fp8 {act}") < 1e-2

@@ -124,3 +124,36 @@ def test_planted_mistakes_are_caught(golden):
     np.testing.assert_allclose(right[0], g["out"], rtol=1e-14, atol=1e-14)
     for bad in (swapped, dropped):
         assert not np.allclose(bad[0], g["out"])
+
+
+def test_gated_activations_match_torch():
+    z = np.linspace(-12, 12, 20001)
+    t = torch.from_numpy(z)
+    np.testing.assert_allclose(O.silu(z), torch.nn.functional.silu(t).numpy(), rtol=1e-14, atol=1e-300)
+    np.testing.assert_allclose(O.gelu(z), torch.nn.functional.gelu(t).numpy(), rtol=1e-13, atol=1e-15)
+    assert np.array_equal(O.relu(z), torch.relu(t).numpy())
+    # closed forms: gelu(0) = 0, gelu(x) -> x for large x, Phi(1) = (1 + erf(1/sqrt 2)) / 2
+    assert O.gelu(0.0) == 0.0 and abs(O.gelu(40.0) - 40.0) < 1e-12
+    assert abs(O.gelu(1.0) - 0.8413447460685429) < 1e-15
+    assert O.relu(-1.0) == 0.0 and O.relu(2.5) == 2.5
+
+
+@pytest.mark.parametrize("act", ["gelu", "relu"])
+def test_gated_activation_forward_matches_batched(act):
+    rng = np.random.default_rng(9)
+    T, H, I, E, k = 12, 32, 48, 5, 2
+    x = rng.standard_normal((T, H))
+    L = rng.standard_normal((T, E), dtype=np.float32)
+    idx, w, _ = O.route(L, k)
+    wgu = rng.standard_normal((E, 2 * I, H)) * 0.2
+    wd = rng.standard_normal((E, H, I)) * 0.2
+    out = O.moe_forward(x, idx, w, wgu, wd, intermediate="none", act=act)
+    f = torch.nn.functional.gelu if act == "gelu" else torch.relu
+    ref = np.zeros((T, H))
+    for t in range(T):
+        for j in range(k):
+            e = idx[t, j]
+            xt = torch.from_numpy(x[t])
+            h = f(torch.from_numpy(wgu[e, :I]) @ xt) * (torch.from_numpy(wgu[e, I:]) @ xt)
+            ref[t] += float(w[t, j]) * (torch.from_numpy(wd[e]) @ h).numpy()
+    np.testing.assert_allclose(out, ref, rtol=1e-11, atol=1e-12)
