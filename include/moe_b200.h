@@ -164,6 +164,25 @@ moe_status moe_workspace_query(const moe_shape* shape, moe_workspace_layout* lay
 moe_status moe_read_device_status(const void* workspace, void* stream);
 
 /*
+ * moe_set_test_hooks -- the failure-detection test's switches. Not for
+ * production use; the page has no counterpart.
+ *
+ *  - wait_limit_ns: how long every bounded wait inside the GEMM kernels spins
+ *    before it gives up, records MOE_ERR_DEVICE_TIMEOUT in the status word,
+ *    lets its CTA's copies and MMAs in flight finish, frees its tensor memory
+ *    and returns. 0 restores the default of 2 s; otherwise 1 ms to 60 s.
+ *  - stall_gate_up_loads: 1 makes the prefill gate/up GEMM's producer issue no
+ *    loads, so the MMA issuer waits on a barrier nothing completes and gives up
+ *    after wait_limit_ns; the rest of the call then runs on stale intermediates
+ *    and its output is garbage. 0 turns it off.
+ *
+ * Both are process-wide and read when a call is enqueued; do not change them
+ * while other threads enqueue calls. Returns MOE_ERR_INVALID_ARG (and changes
+ * nothing) for values outside those ranges.
+ */
+moe_status moe_set_test_hooks(int32_t stall_gate_up_loads, uint64_t wait_limit_ns);
+
+/*
  * moe_forward_noalloc -- moe_forward for callers that cannot allocate device
  * memory. The page has no counterpart to this entry point; it exists for
  * callers that are handed only their input and output buffers (a plugin loaded

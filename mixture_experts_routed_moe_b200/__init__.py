@@ -28,7 +28,8 @@ PATH = {"auto": 0, "prefill": 1, "decode": 2}
 ACT = {"silu": 0, "gelu": 1, "relu": 2}
 PATH_NAMES = {v: k for k, v in PATH.items()}
 EXPORTS = ["moe_route", "moe_workspace_size", "moe_forward", "moe_forward_timed", "moe_workspace_query",
-           "moe_read_device_status", "moe_status_string", "moe_version", "moe_forward_noalloc"]
+           "moe_read_device_status", "moe_status_string", "moe_version", "moe_forward_noalloc",
+           "moe_set_test_hooks"]
 
 
 class MoeError(RuntimeError):
@@ -77,6 +78,8 @@ def lib() -> ctypes.CDLL:
         L.moe_status_string.restype = ctypes.c_char_p
         L.moe_forward_noalloc.argtypes = [ctypes.POINTER(MoeShape), vp, vp, vp, vp, vp, vp, vp, vp, vp]
         L.moe_forward_noalloc.restype = i32
+        L.moe_set_test_hooks.argtypes = [i32, ctypes.c_uint64]
+        L.moe_set_test_hooks.restype = i32
         L.moe_version.argtypes = []
         L.moe_version.restype = i32
         _lib = L
@@ -189,6 +192,13 @@ def read_device_status(workspace: torch.Tensor, stream=None) -> int:
     return int(lib().moe_read_device_status(_ptr(workspace), _stream(stream)))
 
 
+def set_test_hooks(stall_gate_up_loads: bool = False, wait_limit_ns: int = 0) -> None:
+    """Failure-detection test switches (moe_set_test_hooks): the limit of every
+    bounded device wait (0 = the 2 s default) and a stall of the prefill
+    gate/up GEMM's loads. Raises MoeError on values out of range."""
+    _check(lib().moe_set_test_hooks(int(bool(stall_gate_up_loads)), int(wait_limit_ns)), "moe_set_test_hooks")
+
+
 class MoELayer:
     """A routed MoE layer whose expert weights live on the GPU: ``layer(x, logits)``
     runs moe_route then moe_forward and returns bf16 [T,H]. The workspace is
@@ -254,5 +264,5 @@ class MoEGraph:
 
 
 __all__ = ["lib", "route", "forward", "forward_noalloc", "MoEGraph", "workspace_size", "workspace_layout", "alloc_workspace",
-           "read_device_status", "make_shape", "MoELayer", "MoeError", "MoeShape", "EXPORTS", "STATUS",
+           "read_device_status", "set_test_hooks", "make_shape", "MoELayer", "MoeError", "MoeShape", "EXPORTS", "STATUS",
            "status_string", "PATH", "WDTYPE", "ACT"]

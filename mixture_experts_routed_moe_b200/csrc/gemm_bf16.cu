@@ -48,6 +48,7 @@ struct GemmParams {
   int act;  // gate activation (moe_activation)
   int* dev_status;
   unsigned long long timeout_ns;
+  int stall_loads;  // failure-detection test: the producer issues nothing
 };
 
 template <int kN>
@@ -119,7 +120,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t ph = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+      for (int tile = blockIdx.x; ok && !p.stall_loads && tile < total; tile += gridDim.x) {
         const TileCoord c = tile_coord(tile, s_mt, s_cnt, p.E, NT);
         const int brow = c.e * p.b_rows_per_expert + c.n * p.b_tile_stride;
         for (int kb = 0; kb < p.num_kb; ++kb) {
@@ -278,7 +279,8 @@ cudaError_t launch_gemm_bf16(const moe_shape* s, const Plan& p, const void* w_ga
   gp.cnt = reinterpret_cast<const int*>(ws + p.cnt);
   gp.E = E;
   gp.dev_status = reinterpret_cast<int*>(ws + p.status);
-  gp.timeout_ns = kDefaultTimeoutNs;
+  gp.timeout_ns = wait_limit_ns();
+  gp.stall_loads = which == 0 && stall_gate_up_loads() ? 1 : 0;
   gp.act = s->act;
   // every tile count is bounded by the row capacity
   const int max_mtiles = static_cast<int>(p.m_rows / kTileM);

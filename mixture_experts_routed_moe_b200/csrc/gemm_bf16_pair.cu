@@ -281,7 +281,7 @@ cudaError_t launch_gemm_bf16_pair(const moe_shape* s, const Plan& p, const void*
   pp.cnt = reinterpret_cast<const int*>(ws + p.cnt);
   pp.E = E;
   pp.dev_status = reinterpret_cast<int*>(ws + p.status);
-  pp.timeout_ns = kDefaultTimeoutNs;
+  pp.timeout_ns = wait_limit_ns();
   // upper bound of the pair-tile count: every expert's pairs fit in (row blocks + E) / 2 + E
   const int max_pairs = static_cast<int>(p.m_rows / kTileM) / 2 + E;
   CUtensorMap tmA, tmB;

@@ -330,7 +330,7 @@ cudaError_t launch_gemm_e4m3(const moe_shape* s, const Plan& p, const void* /*x*
   fp.cnt = reinterpret_cast<const int*>(ws + p.cnt);
   fp.E = E;
   fp.dev_status = reinterpret_cast<int*>(ws + p.status);
-  fp.timeout_ns = kDefaultTimeoutNs;
+  fp.timeout_ns = wait_limit_ns();
   fp.act = s->act;
   const int max_mtiles = static_cast<int>(p.m_rows / kTileM);
   CUtensorMap tmA, tmB;

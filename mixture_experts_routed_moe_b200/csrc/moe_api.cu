@@ -38,6 +38,9 @@ EncodeTiledFn encode_fn() {
 }
 
 constexpr int kMaxDevices = 64;
+
+std::atomic<unsigned long long> g_wait_limit_ns{kDefaultTimeoutNs};
+std::atomic<int> g_stall_gate_up{0};
 std::atomic<int> g_sm_count[kMaxDevices];
 
 }  // namespace
@@ -146,6 +149,9 @@ bool make_plan(const moe_shape* s, Plan* p) {
   p->total = off;
   return true;
 }
+
+unsigned long long wait_limit_ns() { return g_wait_limit_ns.load(std::memory_order_relaxed); }
+bool stall_gate_up_loads() { return g_stall_gate_up.load(std::memory_order_relaxed) != 0; }
 
 }  // namespace moe
 
@@ -269,6 +275,14 @@ moe_status moe_workspace_query(const moe_shape* shape, moe_workspace_layout* lay
   layout->path = p.path;
   layout->m_rows = static_cast<int32_t>(p.m_rows);
   layout->reserved = 0;
+  return MOE_OK;
+}
+
+moe_status moe_set_test_hooks(int32_t stall_gate_up_loads, uint64_t wait_limit_ns) {
+  if (stall_gate_up_loads != 0 && stall_gate_up_loads != 1) return MOE_ERR_INVALID_ARG;
+  if (wait_limit_ns != 0 && (wait_limit_ns < 1000000ull || wait_limit_ns > 60000000000ull)) return MOE_ERR_INVALID_ARG;
+  g_wait_limit_ns.store(wait_limit_ns == 0 ? kDefaultTimeoutNs : wait_limit_ns);
+  g_stall_gate_up.store(stall_gate_up_loads);
   return MOE_OK;
 }
 

@@ -16,6 +16,12 @@ constexpr int kPermuteTokens = 256;  // tokens per block in the permute kernels
 constexpr int kSmallPermuteT = 256;  // T up to this uses the single-block permute
 constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;  // bounded waits give up after 2 s
 
+// Limit of every bounded device wait (kDefaultTimeoutNs unless a test set
+// another through moe_set_test_hooks), and that entry point's switch that makes
+// the gate/up GEMM's producer issue no loads.
+unsigned long long wait_limit_ns();
+bool stall_gate_up_loads();
+
 // Where every intermediate lives inside the caller's workspace.
 struct Plan {
   int path;        // resolved moe_path (PREFILL or DECODE)

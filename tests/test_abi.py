@@ -115,6 +115,16 @@ def test_route_host_errors(L):
     assert L.moe_route(None, 0, 8, 2, None, None, None) == 0
 
 
+def test_test_hooks_validate_and_reset(L):
+    assert L.moe_set_test_hooks(2, 0) == -1
+    assert L.moe_set_test_hooks(0, 999_999) == -1  # below 1 ms
+    assert L.moe_set_test_hooks(0, 60_000_000_001) == -1
+    assert L.moe_set_test_hooks(1, 5_000_000) == 0
+    assert L.moe_set_test_hooks(0, 0) == 0  # back to the defaults
+    with pytest.raises(moe.MoeError):
+        moe.set_test_hooks(wait_limit_ns=10)
+
+
 def test_missing_library_fails_loudly(monkeypatch):
     monkeypatch.setattr(moe, "_lib", None)
     monkeypatch.setattr(moe, "LIB_PATH", "/nonexistent/libmoe_b200.so")
