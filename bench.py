@@ -7,7 +7,7 @@ A step is one pass of the whole hot path on one batch of synthetic input:
 moe_route (router top-k) followed by moe_forward (permute, gate/up with
 SwiGLU, down, combine) of one layer. The default workload is the
 decode-shaped layer (T=16, H=2048, I=1408, E=60, k=4, bf16); --workload picks
-another (tiny, decode, prefill, fp8, skewed).
+another (tiny, decode, prefill, fp8, skewed, fp8_decode).
 
 Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events
 on the launching stream, with a 256 MiB buffer written between steps (outside
@@ -264,12 +264,19 @@ def stage_roofline(wl, path, stage_ms, n_touched, peaks, peak_src):
     s = max((1, 2), key=lambda i: stage_ms[i])
     dur_s = stage_ms[s] / 1e3
     if path == "decode":
+        fp8 = wl.wdtype == "e4m3"
+        # e4m3: one UE8M0 byte per 128x128 weight block, h stored as e4m3 codes
+        s_gu = n_touched * (2 * I // 128) * (H // 128) if fp8 else 0
+        s_d = n_touched * (H // 128) * (I // 128) if fp8 else 0
+        h_bytes = A * I * welem
         if s == 1:
-            byts = n_touched * 2 * I * H * welem + wl.T * H * 2 + A * I * 2
-            kern, src = "decode_gate_up_kernel", "decode.cu"
+            byts = n_touched * 2 * I * H * welem + s_gu + wl.T * H * 2 + h_bytes
+            kern, src = (("decode_e4m3_gate_up_kernel", "decode_e4m3.cu") if fp8
+                         else ("decode_gate_up_kernel", "decode.cu"))
         else:
-            byts = n_touched * H * I * welem + A * I * 2 + A * H * 2
-            kern, src = "decode_down_kernel", "decode.cu"
+            byts = n_touched * H * I * welem + s_d + h_bytes + A * H * 2
+            kern, src = (("decode_e4m3_down_kernel", "decode_e4m3.cu") if fp8
+                         else ("decode_down_kernel", "decode.cu"))
         ach = byts / dur_s / 1e9
         peak = peaks["hbm_gbs"]
         out = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
@@ -381,7 +388,10 @@ def run_ours(args, world, rank, local):
         raise RuntimeError("graph replay and eager forward disagree")
 
     peaks, peak_src = load_peaks()
-    per_step_launches = 1 + (1 if wl.T <= 256 else 3) + 2 + 1  # route, permute, gate/up, down, combine
+    # route, permute, gate/up, down, combine; the e4m3 DECODE path adds the
+    # per-token x quantisation and the h quantisation
+    per_step_launches = (1 + (1 if wl.T <= 256 else 3) + 2 + 1
+                         + (2 if path == "decode" and wl.wdtype == "e4m3" else 0))
     tokens = wl.T * K * world
     value = tokens / (total_ms / 1e3)
     line = {

@@ -52,9 +52,9 @@ typedef enum { MOE_DT_BF16 = 0, MOE_DT_E4M3 = 1 } moe_wdtype;
 /* Which execution of the expert matmuls to use (the page's decode-stage switch:
  * small token counts run better on a per-token form than on grouped GEMM tiles). */
 typedef enum {
-  MOE_PATH_AUTO = 0,    /* DECODE when T*k <= 4*E and weights are bf16, else PREFILL */
+  MOE_PATH_AUTO = 0,    /* DECODE when T*k <= 4*E, else PREFILL */
   MOE_PATH_PREFILL = 1, /* expert-major permute + tcgen05 grouped GEMMs */
-  MOE_PATH_DECODE = 2   /* weight-streaming kernels, no tile padding (bf16 only) */
+  MOE_PATH_DECODE = 2   /* weight-streaming kernels, no tile padding */
 } moe_path;
 
 /* Gate activation of the gated expert MLP (section "SonicMoE": SwiGLU, GeGLU
@@ -120,8 +120,8 @@ size_t moe_workspace_size(const moe_shape* shape);
  * Errors: MOE_ERR_SCALE_FORMAT when wdtype is e4m3 and a scale pointer is NULL
  * (the page's note: Blackwell kernels need UE8M0 scales and refuse plain float
  * ones instead of silently corrupting the output); MOE_ERR_UNSUPPORTED for
- * MOE_PATH_DECODE with e4m3 weights and for e4m3 weights with H not a multiple
- * of 256.
+ * e4m3 weights on the PREFILL path with H not a multiple of 256 (the DECODE
+ * path takes any H that is a multiple of 128).
  */
 moe_status moe_forward(const moe_shape* shape, const void* x, const int32_t* topk_idx,
                        const float* topk_w, const void* w_gate_up, const void* w_down,
@@ -145,8 +145,10 @@ moe_status moe_forward_timed(const moe_shape* shape, const void* x, const int32_
  *   mt_base   int32 [E+1]  expert e owns rows [mt_base[e]*bm, mt_base[e+1]*bm)
  *   row_src   int32 [m_rows] assignment t*k+j held by each row, -1 for padding
  *   slot_row  int32 [T*k]  row of assignment t*k+j
- *   xa        permuted activations (PREFILL): bf16 [m_rows, H] or e4m3 [m_rows, H]
- *   xs        fp32 [m_rows, H/128] activation scales (e4m3 only)
+ *   xa        permuted activations: bf16 [m_rows, H] (bf16 PREFILL only), e4m3
+ *             codes [m_rows, H] (e4m3 PREFILL) or e4m3 codes [T, H] in token
+ *             order (e4m3 DECODE: each token quantised once)
+ *   xs        fp32 activation scales [rows of xa, H/128] (e4m3 only)
  *   h         bf16 [m_rows, I] (or e4m3 with fp32 scales hs [m_rows, I/128])
  *   y         bf16 [m_rows, H] expert outputs
  * m_rows is the allocated row capacity; only rows below mt_base[E]*bm are used.

@@ -61,12 +61,6 @@ struct Fp8Params {
   unsigned long long timeout_ns;
 };
 
-__device__ __forceinline__ float ue8m0_value(uint32_t b) {
-  if (b == 0) return 5.877471754111438e-39f;  // 2^-127 (subnormal)
-  if (b == 255) return __int_as_float(0x7fc00000);
-  return __int_as_float(b << 23);
-}
-
 __device__ __forceinline__ void epi_bar_sync() { asm volatile("bar.sync 1, %0;" ::"n"(32 * kEpiWarps) : "memory"); }
 
 template <bool kGateUp>

@@ -103,7 +103,7 @@ bool validate_shape(const moe_shape* s) {
 
 int resolve_path(const moe_shape* s) {
   if (s->path != MOE_PATH_AUTO) return s->path;
-  if (s->wdtype == MOE_DT_BF16 && static_cast<long long>(s->T) * s->k <= 4ll * s->E && decode_supported(s))
+  if (static_cast<long long>(s->T) * s->k <= 4ll * s->E && decode_supported(s))
     return MOE_PATH_DECODE;
   return MOE_PATH_PREFILL;
 }
@@ -141,10 +141,15 @@ bool make_plan(const moe_shape* s, Plan* p) {
   p->row_src = take(std::max<size_t>(M, 1) * 4);
   p->slot_row = take(std::max<long long>(A, 1) * 4);
   const size_t act = fp8 ? 1 : 2;
-  p->xa = (p->path == MOE_PATH_PREFILL) ? take(M * H * act) : none;
-  p->xs = (p->path == MOE_PATH_PREFILL && fp8) ? take(M * (H / 128) * 4) : none;
+  // permuted x: bf16 copy (bf16 PREFILL) or e4m3 codes (both e4m3 paths);
+  // bf16 DECODE reads the token rows of x in place
+  // (e4m3 DECODE: one row per token, not per assignment)
+  const size_t xrows = (fp8 && p->path == MOE_PATH_DECODE) ? static_cast<size_t>(T) : M;
+  p->xa = (p->path == MOE_PATH_PREFILL || fp8) ? take(xrows * H * act) : none;
+  p->xs = fp8 ? take(xrows * (H / 128) * 4) : none;
   p->h = take(M * I * act);
   p->hs = fp8 ? take(M * (I / 128) * 4) : none;
+  p->hf = (fp8 && p->path == MOE_PATH_DECODE) ? take(M * I * 4) : none;
   p->y = take(M * H * 2);
   p->total = off;
   return true;
@@ -169,8 +174,8 @@ moe_status forward_impl(const moe_shape* shape, const void* x, const int32_t* to
   if (fp8 && (sw_gate_up == nullptr || sw_down == nullptr)) return MOE_ERR_SCALE_FORMAT;
   Plan plan;
   if (!make_plan(shape, &plan)) return MOE_ERR_INVALID_ARG;
-  // e4m3 experts: PREFILL only, and the down tile spans two 128-column scale blocks
-  if (fp8 && (plan.path == MOE_PATH_DECODE || !e4m3_path_available() || shape->H % 256 != 0))
+  // e4m3 PREFILL: the down tile spans two 128-column scale blocks
+  if (fp8 && plan.path == MOE_PATH_PREFILL && (!e4m3_path_available() || shape->H % 256 != 0))
     return MOE_ERR_UNSUPPORTED;
   if (plan.path == MOE_PATH_DECODE && !decode_supported(shape)) return MOE_ERR_UNSUPPORTED;
   if (shape->T == 0) return MOE_OK;
@@ -194,7 +199,11 @@ moe_status forward_impl(const moe_shape* shape, const void* x, const int32_t* to
   if (launch_permute(shape, plan, topk_idx, x, ws, st) != cudaSuccess) return MOE_ERR_CUDA;
   if (!mark(1)) return MOE_ERR_CUDA;
   cudaError_t err;
-  if (plan.path == MOE_PATH_DECODE) {
+  if (plan.path == MOE_PATH_DECODE && fp8) {
+    err = launch_decode_e4m3(shape, plan, w_gate_up, w_down, sw_gate_up, sw_down, ws, 0, sms, st);
+    if (err != cudaSuccess || !mark(2)) return MOE_ERR_CUDA;
+    err = launch_decode_e4m3(shape, plan, w_gate_up, w_down, sw_gate_up, sw_down, ws, 1, sms, st);
+  } else if (plan.path == MOE_PATH_DECODE) {
     err = launch_decode(shape, plan, x, w_gate_up, w_down, ws, 0, sms, st);
     if (err != cudaSuccess || !mark(2)) return MOE_ERR_CUDA;
     err = launch_decode(shape, plan, x, w_gate_up, w_down, ws, 1, sms, st);

@@ -320,6 +320,24 @@ __device__ __forceinline__ float gated_act(int act, float g, float u) {
 }
 
 // Streaming 16-byte load that does not allocate in L1.
+// UE8M0 block scale byte b -> 2^(b-127) (255 is NaN in the format).
+__device__ __forceinline__ float ue8m0_value(uint32_t b) {
+  if (b == 0) return 5.877471754111438e-39f;  // 2^-127 (subnormal)
+  if (b == 255) return __int_as_float(0x7fc00000);
+  return __int_as_float(b << 23);
+}
+
+// Four e4m3 codes (one 32-bit word, lowest byte first) -> fp32, exactly.
+__device__ __forceinline__ void e4m3x4_to_f32(uint32_t v, float* f) {
+  const __half2 lo = __half2(__nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(v & 0xFFFFu), __NV_E4M3));
+  const __half2 hi = __half2(__nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(v >> 16), __NV_E4M3));
+  const float2 a = __half22float2(lo), b = __half22float2(hi);
+  f[0] = a.x;
+  f[1] = a.y;
+  f[2] = b.x;
+  f[3] = b.y;
+}
+
 __device__ __forceinline__ uint4 ld_stream_u4(const void* p) {
   uint4 v;
   asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"

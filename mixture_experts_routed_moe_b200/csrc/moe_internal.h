@@ -29,7 +29,7 @@ struct Plan {
   int64_t m_rows;  // row capacity of the permuted buffers
   int nblk;        // permute blocks of kPermuteTokens tokens
   size_t status, hdr, block_counts, cnt, mt_base, pt_base, touched, local_rank, row_src, slot_row;
-  size_t xa, xs, h, hs, y, total;
+  size_t xa, xs, h, hs, hf, y, total;  // hf: fp32 h of the e4m3 DECODE path
 };
 
 // Header words written on the device by the permute stage.
@@ -61,6 +61,11 @@ bool e4m3_path_available();
 bool decode_supported(const moe_shape* s);
 cudaError_t launch_decode(const moe_shape* s, const Plan& p, const void* x, const void* w_gate_up,
                           const void* w_down, uint8_t* ws, int which, int num_sms, cudaStream_t st);
+// e4m3 experts on the DECODE path: which = 0 runs gate/up and the h
+// quantisation, which = 1 the down projection.
+cudaError_t launch_decode_e4m3(const moe_shape* s, const Plan& p, const void* w_gate_up, const void* w_down,
+                               const uint8_t* sw_gate_up, const uint8_t* sw_down, uint8_t* ws, int which,
+                               int num_sms, cudaStream_t st);
 
 cudaError_t launch_combine(const moe_shape* s, const Plan& p, const float* topk_w, void* out, uint8_t* ws,
                            cudaStream_t st);

@@ -15,6 +15,8 @@
 // population count of the masks of earlier warps plus the bits of earlier
 // lanes in its own warp, and blocks are offset by an exclusive scan of the
 // per-block counts.
+#include <algorithm>
+
 #include "moe_common.cuh"
 #include "moe_internal.h"
 
@@ -22,6 +24,9 @@ namespace moe {
 namespace {
 
 constexpr int kWarps = kPermuteTokens / 32;  // 8 warps, one token per thread
+// the single-block permute stages rows itself up to this many elements (a few
+// loads per warp); larger volumes go to stage_rows_kernel
+constexpr long long kSmallStageElems = 32768;
 
 // Phase 1 of the block-level count: per-warp expert masks in shared memory.
 // Records kDevErrIndex for an index outside [0,E) or a repeated expert.
@@ -153,37 +158,77 @@ __device__ __forceinline__ void copy_row_bf16(const __nv_bfloat16* __restrict__ 
   for (int c = lane; c < H / 8; c += 32) dst[c] = __ldg(src + c);
 }
 
-// Quantise one assignment's hidden-state row into its permuted row (one warp):
-// per 128-column group, scale s = amax/448 in fp32 (1 for an all-zero group)
-// and codes e4m3(x/s), round to nearest even, saturating (the FP8 experts'
-// dynamic per-row activation scales). Each half-warp owns one group at a time.
+// Quantise one 128-column group of a bf16 row with one half-warp (lane l16
+// holds columns 8*l16 .. 8*l16+7, in v): scale s = amax/448 in fp32 (1 for
+// an all-zero group) and codes e4m3(x/s) with IEEE division, round to nearest
+// even, saturating -- the FP8 experts' dynamic per-row activation scales.
+__device__ __forceinline__ void quant_group_e4m3(const uint4& v, unsigned hmask, int l16, uint2* dst, float* scale) {
+  const float f[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
+                      bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(hmask, amax, o));
+  const float sc = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+  uint32_t w[2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(__fdiv_rn(f[4 * i], sc), __fdiv_rn(f[4 * i + 1], sc)),
+                                                 __NV_SATFINITE, __NV_E4M3);
+    const uint32_t hi = __nv_cvt_float2_to_fp8x2(
+        make_float2(__fdiv_rn(f[4 * i + 2], sc), __fdiv_rn(f[4 * i + 3], sc)), __NV_SATFINITE, __NV_E4M3);
+    w[i] = lo | (hi << 16);
+  }
+  *dst = make_uint2(w[0], w[1]);
+  if (l16 == 0) *scale = sc;
+}
+
+// Quantise one token's row into permuted row `row` (one warp; each half-warp
+// owns one group at a time).
 __device__ __forceinline__ void quant_row_e4m3(const __nv_bfloat16* __restrict__ x, uint8_t* __restrict__ xq,
                                                float* __restrict__ xs, int t, int row, int H, int lane) {
   const int half = lane >> 4, l16 = lane & 15;
   const unsigned hmask = 0xFFFFu << (16 * half);
   const int G = H / 128;
   const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H);
-  for (int g = half; g < G; g += 2) {
-    const uint4 v = __ldg(src + g * 16 + l16);
-    const float f[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
-                        bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
-    float amax = 0.f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
-#pragma unroll
-    for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(hmask, amax, o));
-    const float sc = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
-    uint32_t w[2];
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(__fdiv_rn(f[4 * i], sc), __fdiv_rn(f[4 * i + 1], sc)),
-                                                   __NV_SATFINITE, __NV_E4M3);
-      const uint32_t hi = __nv_cvt_float2_to_fp8x2(
-          make_float2(__fdiv_rn(f[4 * i + 2], sc), __fdiv_rn(f[4 * i + 3], sc)), __NV_SATFINITE, __NV_E4M3);
-      w[i] = lo | (hi << 16);
+  for (int g = half; g < G; g += 2)
+    quant_group_e4m3(__ldg(src + g * 16 + l16), hmask, l16,
+                     reinterpret_cast<uint2*>(xq + static_cast<size_t>(row) * H + g * 128) + l16,
+                     xs + static_cast<size_t>(row) * G + g);
+}
+
+// Copies (bf16, into xa) or quantises (e4m3, into xq/xs) activation rows, one
+// half-warp per (source, 128-column group) task spread over many blocks, so
+// the row traffic is not left to the single block of the small permute.
+// With slot_row the sources are assignments a (token a / k, destination row
+// slot_row[a], skipped when negative); without it they are tokens, each
+// written once to row t (the e4m3 DECODE path reads x per token).
+__global__ void __launch_bounds__(256) stage_rows_kernel(const __nv_bfloat16* __restrict__ x,
+                                                         const int* __restrict__ slot_row, long long n_src, int k,
+                                                         int H, __nv_bfloat16* __restrict__ xa,
+                                                         uint8_t* __restrict__ xq, float* __restrict__ xs) {
+  const int G = H / 128;
+  const long long total = n_src * G;
+  const int l16 = threadIdx.x & 15;
+  const unsigned hmask = 0xFFFFu << (threadIdx.x & 16);
+  const long long stride = static_cast<long long>(gridDim.x) * (blockDim.x / 16);
+  for (long long task = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) / 16; task < total;
+       task += stride) {
+    const long long a = task / G;
+    const int g = static_cast<int>(task - a * G);
+    long long row = a, t = a;
+    if (slot_row != nullptr) {
+      row = slot_row[a];
+      t = a / k;
+      if (row < 0) continue;  // the whole half-warp skips together
     }
-    *reinterpret_cast<uint2*>(xq + static_cast<size_t>(row) * H + g * 128 + l16 * 8) = make_uint2(w[0], w[1]);
-    if (l16 == 0) xs[static_cast<size_t>(row) * G + g] = sc;
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H + g * 128) + l16);
+    if (xa != nullptr)
+      reinterpret_cast<uint4*>(xa + static_cast<size_t>(row) * H + g * 128)[l16] = v;
+    else
+      quant_group_e4m3(v, hmask, l16, reinterpret_cast<uint2*>(xq + static_cast<size_t>(row) * H + g * 128) + l16,
+                       xs + static_cast<size_t>(row) * G + g);
   }
 }
 
@@ -306,32 +351,50 @@ cudaError_t launch_permute(const moe_shape* s, const Plan& p, const int* topk_id
   int* lrank = reinterpret_cast<int*>(ws + p.local_rank);
   int* row_src = reinterpret_cast<int*>(ws + p.row_src);
   int* slot_row = reinterpret_cast<int*>(ws + p.slot_row);
-  // the permuted bf16 copy of x is only needed by the bf16 PREFILL path
-  __nv_bfloat16* xa = (p.path == MOE_PATH_PREFILL && s->wdtype == MOE_DT_BF16)
-                          ? reinterpret_cast<__nv_bfloat16*>(ws + p.xa)
-                          : nullptr;
-  // the e4m3 PREFILL path quantises x into its permuted rows instead
-  uint8_t* xq = (p.path == MOE_PATH_PREFILL && s->wdtype == MOE_DT_E4M3) ? ws + p.xa : nullptr;
-  float* xs = xq != nullptr ? reinterpret_cast<float*>(ws + p.xs) : nullptr;
+  const bool fp8 = s->wdtype == MOE_DT_E4M3;
+  const bool prefill = p.path == MOE_PATH_PREFILL;
+  // PREFILL: x copied (bf16) or quantised (e4m3) into the permuted rows;
+  // e4m3 DECODE: x quantised once per token; bf16 DECODE reads x in place
+  __nv_bfloat16* xa = (prefill && !fp8) ? reinterpret_cast<__nv_bfloat16*>(ws + p.xa) : nullptr;
+  uint8_t* xq = fp8 ? ws + p.xa : nullptr;
+  float* xs = fp8 ? reinterpret_cast<float*>(ws + p.xs) : nullptr;
   const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
   const size_t mask_bytes = sizeof(uint32_t) * kWarps * E;
+  const long long A = static_cast<long long>(T) * k;
+  const int G = H / 128;
+  // rows are staged by the permute kernels themselves only where that is
+  // short: the single-block permute for at most kSmallStageElems elements
+  const bool stage_in_small = prefill && A * H <= kSmallStageElems;
+  auto stage = [&](const int* slots, long long n_src) -> cudaError_t {
+    const long long tasks = n_src * G;
+    const long long want = (tasks + 15) / 16;  // blocks of 16 half-warps
+    const long long cap = static_cast<long long>(device_sm_count()) * 8;
+    const unsigned grid = static_cast<unsigned>(std::max<long long>(1, std::min(want, cap)));
+    stage_rows_kernel<<<grid, 256, 0, st>>>(xb, slots, n_src, k, H, xa, xq, xs);
+    return cudaGetLastError();
+  };
 
   cudaError_t err = cudaMemsetAsync(status, 0, sizeof(int), st);
   if (err != cudaSuccess) return err;
   if (T <= kSmallPermuteT) {
     permute_small_kernel<<<1, 1024, mask_bytes, st>>>(topk_idx, T, k, E, p.bm, cnt, mt_base, pt_base, touched, hdr,
-                                                      row_src,
-                                                      slot_row, lrank, status, xb, xa, xq, xs, H);
-    return cudaGetLastError();
+                                                      row_src, slot_row, lrank, status, xb,
+                                                      stage_in_small ? xa : nullptr,
+                                                      stage_in_small ? xq : nullptr,
+                                                      stage_in_small ? xs : nullptr, H);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    if (stage_in_small || (!prefill && !fp8)) return cudaSuccess;
+    return prefill ? stage(slot_row, A) : stage(nullptr, T);
   }
   permute_count_kernel<<<p.nblk, kPermuteTokens, mask_bytes, st>>>(topk_idx, T, k, E, counts, lrank, status);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   permute_scan_kernel<<<1, 1024, 0, st>>>(counts, p.nblk, E, p.bm, cnt, mt_base, pt_base, touched, hdr, row_src);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
-  const long long A = static_cast<long long>(T) * k;
   permute_scatter_kernel<<<static_cast<unsigned>((A + 7) / 8), 256, 0, st>>>(
-      topk_idx, T, k, E, p.bm, counts, lrank, mt_base, row_src, slot_row, xb, xa, xq, xs, H);
-  return cudaGetLastError();
+      topk_idx, T, k, E, p.bm, counts, lrank, mt_base, row_src, slot_row, xb, xa, prefill ? xq : nullptr,
+      prefill ? xs : nullptr, H);
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  return (!prefill && fp8) ? stage(nullptr, T) : cudaSuccess;
 }
 
 }  // namespace moe

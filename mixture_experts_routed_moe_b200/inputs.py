@@ -73,9 +73,11 @@ WORKLOADS = {
     "prefill": Workload("prefill", 8192, 2048, 768, 128, 8),
     "fp8": Workload("fp8", 4096, 7168, 2048, 256, 8, wdtype="e4m3"),
     "skewed": Workload("skewed", 4096, 4096, 14336, 8, 2, router_bias=True),
+    # the FP8 layer's experts at decode size: 16 tokens, weight-streaming path
+    "fp8_decode": Workload("fp8_decode", 16, 7168, 2048, 256, 8, wdtype="e4m3"),
 }
 # the seed of each named workload is its position in this list
-WORKLOAD_ORDER = ["tiny", "decode", "prefill", "fp8", "skewed"]
+WORKLOAD_ORDER = ["tiny", "decode", "prefill", "fp8", "skewed", "fp8_decode"]
 
 
 def default_seed(wl: Workload) -> int:

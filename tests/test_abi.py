@@ -77,7 +77,8 @@ def test_workspace_layout_is_consistent(L):
 def test_auto_path_choice(L):
     assert moe.workspace_layout(shape(T=16, H=2048, I=1408, E=60, k=4)).path == moe.PATH["decode"]
     assert moe.workspace_layout(shape(T=8192, H=2048, I=768, E=128, k=8)).path == moe.PATH["prefill"]
-    assert moe.workspace_layout(shape(T=16, E=60, k=4, wdtype="e4m3")).path == moe.PATH["prefill"]
+    assert moe.workspace_layout(shape(T=16, E=60, k=4, wdtype="e4m3")).path == moe.PATH["decode"]
+    assert moe.workspace_layout(shape(T=4096, E=60, k=4, wdtype="e4m3")).path == moe.PATH["prefill"]
 
 
 def test_scale_format_error_and_host_errors(L):
@@ -85,7 +86,8 @@ def test_scale_format_error_and_host_errors(L):
     # FP8 experts without UE8M0 scales: refused loudly
     r = L.moe_forward(ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, FAKE, None, None, FAKE, FAKE, 1 << 40, None)
     assert r == -3
-    s = shape(wdtype="e4m3", path="decode")
+    # e4m3 PREFILL with H not a multiple of 256: refused before any launch
+    s = shape(wdtype="e4m3", path="prefill", H=384)
     r = L.moe_forward(ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 40, None)
     assert r == -2
     s = shape()
