@@ -282,21 +282,41 @@ def stage_roofline(wl, path, stage_ms, n_touched, peaks, peak_src):
         out = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
                "kernel": kern, "stage": names[s], "algorithmic_bytes": byts}
     else:
+        # the stage is bound by the tensor pipe or by HBM, whichever takes
+        # longer at its measured peak: bf16 prefill shapes are tensor-bound,
+        # the FP8 layer (256 experts, ~128 rows each) streams ~11 GB of weights
+        # and is HBM-bound
         flops = (4 if s == 1 else 2) * A * H * I
-        ach = flops / dur_s / 1e12
-        if wl.wdtype == "e4m3":
-            peak, how = 2.0 * peaks["bf16_tflops"], "2x measured bf16 (nominal fp8:bf16 ratio)"
-            kern, src = ("gemm_e4m3_gate_up" if s == 1 else "gemm_e4m3_down"), "gemm_e4m3.cu"
+        fp8 = wl.wdtype == "e4m3"
+        if s == 1:
+            byts = (n_touched * 2 * I * H * welem + A * H * welem + A * I * welem
+                    + (n_touched * (2 * I // 128) * (H // 128) + A * (H // 128) * 4 + A * (I // 128) * 4 if fp8 else 0))
         else:
-            peak, how = peaks["bf16_tflops"], "measured bf16 burst"
+            byts = (n_touched * H * I * welem + A * I * welem + A * H * 2
+                    + (n_touched * (H // 128) * (I // 128) + A * (I // 128) * 4 if fp8 else 0))
+        if fp8:
+            tpeak, how = 2.0 * peaks["bf16_tflops"], "2x measured bf16 (nominal fp8:bf16 ratio)"
+            kern, src = ("grouped_gemm_e4m3_kernel<true>" if s == 1 else "grouped_gemm_e4m3_kernel<false>"), \
+                "gemm_e4m3.cu"
+        else:
+            tpeak, how = peaks["bf16_tflops"], "measured bf16 burst"
             # gate/up: single-CTA kernel; down: the CTA-pair kernel when H % 256 == 0
             if s == 1:
                 kern, src = "grouped_gemm_bf16_kernel<256,true>", "gemm_bf16.cu"
             else:
                 kern, src = (("grouped_gemm_bf16_pair_kernel", "gemm_bf16_pair.cu") if H % 256 == 0
                              else ("grouped_gemm_bf16_kernel<128,false>", "gemm_bf16.cu"))
-        out = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
-               "kernel": kern, "stage": names[s], "algorithmic_flops": flops, "peak_source": how}
+        t_tensor = flops / (tpeak * 1e12)
+        t_hbm = byts / (peaks["hbm_gbs"] * 1e9)
+        if t_tensor >= t_hbm:
+            ach = flops / dur_s / 1e12
+            out = {"bound": "tensor", "achieved": ach, "peak": tpeak, "unit": "TFLOP/s", "frac": ach / tpeak,
+                   "peak_source": how}
+        else:
+            ach = byts / dur_s / 1e9
+            out = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                   "frac": ach / peaks["hbm_gbs"], "tensor_frac": flops / dur_s / 1e12 / tpeak}
+        out.update({"kernel": kern, "stage": names[s], "algorithmic_flops": flops, "algorithmic_bytes": byts})
     rec = NCU_TRAFFIC.get((wl.name, kern))
     out["traffic"] = rec["bytes"] if rec and rec["src"] == src_hash(src) else None
     out["peak_from"] = peak_src

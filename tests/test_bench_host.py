@@ -58,6 +58,21 @@ def test_roofline_arithmetic():
     r = bench.stage_roofline(wl, "prefill", {1: 0.3, 2: 0.2}, 128, peaks, "measured")
     assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
     assert abs(r["achieved"] - 4 * wl.A * wl.H * wl.I / 3e-4 / 1e12) < 1e-6 * r["achieved"]
+    # the FP8 layer streams more weight bytes than its FLOPs need at the fp8
+    # peak: bound by HBM, algorithmic bytes = touched weights + scales + x + h
+    wl = G.WORKLOADS["fp8"]
+    r = bench.stage_roofline(wl, "prefill", {1: 2.0, 2: 1.0}, 256, peaks, "measured")
+    H, I, A = wl.H, wl.I, wl.A
+    byts = 256 * 2 * I * H + A * H + A * I + 256 * (2 * I // 128) * (H // 128) + A * (H // 128) * 4 + A * (I // 128) * 4
+    assert r["bound"] == "hbm" and r["stage"] == "gate_up" and r["unit"] == "GB/s"
+    assert abs(r["achieved"] - byts / 2e-3 / 1e9) < 1e-6 * r["achieved"]
+    assert 4 * A * H * I / (3000.0 * 1e12) < byts / (6000.0 * 1e9)
+    # e4m3 decode: weight codes plus one scale byte per 128x128 block
+    wl = G.WORKLOADS["fp8_decode"]
+    r = bench.stage_roofline(wl, "decode", {1: 0.5, 2: 0.25}, 90, peaks, "measured")
+    byts = 90 * 2 * wl.I * wl.H + 90 * (2 * wl.I // 128) * (wl.H // 128) + wl.T * wl.H * 2 + wl.A * wl.I
+    assert r["kernel"] == "decode_e4m3_gate_up_kernel"
+    assert abs(r["achieved"] - byts / 5e-4 / 1e9) < 1e-6 * r["achieved"]
 
 
 def test_reference_arm_runs_on_cpu():
