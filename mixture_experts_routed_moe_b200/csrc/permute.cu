@@ -162,7 +162,7 @@ __device__ __forceinline__ void copy_row_bf16(const __nv_bfloat16* __restrict__ 
 // holds columns 8*l16 .. 8*l16+7, in v): scale s = amax/448 in fp32 (1 for
 // an all-zero group) and codes e4m3(x/s) with IEEE division, round to nearest
 // even, saturating -- the FP8 experts' dynamic per-row activation scales.
-__device__ __forceinline__ void quant_group_e4m3(const uint4& v, unsigned hmask, int l16, uint2* dst, float* scale) {
+__device__ __forceinline__ uint2 quant_group_codes(const uint4& v, unsigned hmask, float* sc_out) {
   const float f[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
                       bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
   float amax = 0.f;
@@ -180,7 +180,13 @@ __device__ __forceinline__ void quant_group_e4m3(const uint4& v, unsigned hmask,
         make_float2(__fdiv_rn(f[4 * i + 2], sc), __fdiv_rn(f[4 * i + 3], sc)), __NV_SATFINITE, __NV_E4M3);
     w[i] = lo | (hi << 16);
   }
-  *dst = make_uint2(w[0], w[1]);
+  *sc_out = sc;
+  return make_uint2(w[0], w[1]);
+}
+
+__device__ __forceinline__ void quant_group_e4m3(const uint4& v, unsigned hmask, int l16, uint2* dst, float* scale) {
+  float sc;
+  *dst = quant_group_codes(v, hmask, &sc);
   if (l16 == 0) *scale = sc;
 }
 
@@ -232,9 +238,11 @@ __global__ void __launch_bounds__(256) stage_rows_kernel(const __nv_bfloat16* __
   }
 }
 
-// One warp per assignment: writes row_src / slot_row and, when xa is given,
-// copies the token's hidden state into the permuted row (or, when xq is given,
-// quantises it to e4m3 with per-group scales in xs).
+// One warp per token: writes row_src / slot_row of the token's k assignments
+// and, when xa is given, copies the token's hidden state into each of their
+// permuted rows (or, when xq is given, quantises it once and writes the codes
+// and group scales to each row). The token row is read once per 32
+// assignments, not once per assignment.
 __global__ void __launch_bounds__(256) permute_scatter_kernel(const int* __restrict__ idx, int T, int k, int E, int bm,
                                                               const int* __restrict__ block_base,
                                                               const int* __restrict__ local_rank,
@@ -244,22 +252,56 @@ __global__ void __launch_bounds__(256) permute_scatter_kernel(const int* __restr
                                                               __nv_bfloat16* __restrict__ xa, uint8_t* __restrict__ xq,
                                                               float* __restrict__ xs, int H) {
   const int lane = threadIdx.x & 31;
-  const long long a = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
-  if (a >= static_cast<long long>(T) * k) return;
-  const int t = static_cast<int>(a / k);
-  const int e = idx[a];
-  if (static_cast<unsigned>(e) >= static_cast<unsigned>(E)) {
-    if (lane == 0) slot_row[a] = -1;
-    return;
+  const long long t = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (t >= T) return;
+  const int b = static_cast<int>(t / kPermuteTokens);
+  const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H);
+  const int G = H / 128;
+  const int half = lane >> 4, l16 = lane & 15;
+  const unsigned hmask = 0xFFFFu << (16 * half);
+  for (int j0 = 0; j0 < k; j0 += 32) {
+    const int nj = min(32, k - j0);
+    int row = -1;
+    if (lane < nj) {
+      const long long a = t * k + j0 + lane;
+      const int e = idx[a];
+      if (static_cast<unsigned>(e) < static_cast<unsigned>(E)) {
+        row = mt_base[e] * bm + block_base[static_cast<size_t>(b) * E + e] + local_rank[a];
+        row_src[row] = static_cast<int>(a);
+      }
+      slot_row[a] = row;
+    }
+    if (xa != nullptr) {
+      // uniform trip count (H/8 need not be a multiple of 32): every lane
+      // reaches the full-warp row broadcasts
+      const int nc = H / 8;
+      for (int c0 = 0; c0 < nc; c0 += 32) {
+        const int c = c0 + lane;
+        const uint4 v = c < nc ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
+        for (int j = 0; j < nj; ++j) {
+          const int r = __shfl_sync(0xffffffffu, row, j);
+          if (r >= 0 && c < nc) reinterpret_cast<uint4*>(xa + static_cast<size_t>(r) * H)[c] = v;
+        }
+      }
+    }
+    if (xq != nullptr) {
+      // both half-warps run the same number of iterations (G rounded up to
+      // even), so the full-warp row broadcasts below stay converged
+      for (int g0 = 0; g0 < G; g0 += 2) {
+        const int g = g0 + half;
+        uint2 codes = make_uint2(0u, 0u);
+        float sc = 1.f;
+        if (g < G) codes = quant_group_codes(__ldg(src + g * 16 + l16), hmask, &sc);
+        for (int j = 0; j < nj; ++j) {
+          const int r = __shfl_sync(0xffffffffu, row, j);
+          if (r >= 0 && g < G) {
+            reinterpret_cast<uint2*>(xq + static_cast<size_t>(r) * H + g * 128)[l16] = codes;
+            if (l16 == 0) xs[static_cast<size_t>(r) * G + g] = sc;
+          }
+        }
+      }
+    }
   }
-  const int b = t / kPermuteTokens;
-  const int row = mt_base[e] * bm + block_base[static_cast<size_t>(b) * E + e] + local_rank[a];
-  if (lane == 0) {
-    row_src[row] = static_cast<int>(a);
-    slot_row[a] = row;
-  }
-  if (xa != nullptr) copy_row_bf16(x, xa, t, row, H, lane);
-  if (xq != nullptr) quant_row_e4m3(x, xq, xs, t, row, H, lane);
 }
 
 // Everything in one block of 1024 threads, for T <= kPermuteTokens.
@@ -390,7 +432,7 @@ cudaError_t launch_permute(const moe_shape* s, const Plan& p, const int* topk_id
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   permute_scan_kernel<<<1, 1024, 0, st>>>(counts, p.nblk, E, p.bm, cnt, mt_base, pt_base, touched, hdr, row_src);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
-  permute_scatter_kernel<<<static_cast<unsigned>((A + 7) / 8), 256, 0, st>>>(
+  permute_scatter_kernel<<<static_cast<unsigned>((T + 7) / 8), 256, 0, st>>>(
       topk_idx, T, k, E, p.bm, counts, lrank, mt_base, row_src, slot_row, xb, xa, prefill ? xq : nullptr,
       prefill ? xs : nullptr, H);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
