@@ -275,9 +275,11 @@ __global__ void __launch_bounds__(256) permute_scatter_kernel(const int* __restr
       // uniform trip count (H/8 need not be a multiple of 32): every lane
       // reaches the full-warp row broadcasts
       const int nc = H / 8;
+      uint4 vn = lane < nc ? __ldg(src + lane) : make_uint4(0u, 0u, 0u, 0u);
       for (int c0 = 0; c0 < nc; c0 += 32) {
         const int c = c0 + lane;
-        const uint4 v = c < nc ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
+        const uint4 v = vn;  // the next chunk's load is in flight while this one is stored
+        if (c + 32 < nc) vn = __ldg(src + c + 32);
         for (int j = 0; j < nj; ++j) {
           const int r = __shfl_sync(0xffffffffu, row, j);
           if (r >= 0 && c < nc) reinterpret_cast<uint4*>(xa + static_cast<size_t>(r) * H)[c] = v;
@@ -287,11 +289,14 @@ __global__ void __launch_bounds__(256) permute_scatter_kernel(const int* __restr
     if (xq != nullptr) {
       // both half-warps run the same number of iterations (G rounded up to
       // even), so the full-warp row broadcasts below stay converged
+      uint4 vn = half < G ? __ldg(src + half * 16 + l16) : make_uint4(0u, 0u, 0u, 0u);
       for (int g0 = 0; g0 < G; g0 += 2) {
         const int g = g0 + half;
+        const uint4 v = vn;  // the next group's load is in flight while this one is quantised
+        if (g + 2 < G) vn = __ldg(src + (g + 2) * 16 + l16);
         uint2 codes = make_uint2(0u, 0u);
         float sc = 1.f;
-        if (g < G) codes = quant_group_codes(__ldg(src + g * 16 + l16), hmask, &sc);
+        if (g < G) codes = quant_group_codes(v, hmask, &sc);
         for (int j = 0; j < nj; ++j) {
           const int r = __shfl_sync(0xffffffffu, row, j);
           if (r >= 0 && g < G) {
