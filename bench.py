@@ -52,10 +52,15 @@ DEFAULT_WORKLOAD = "decode"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FLUSH_BYTES = 256 << 20
 
-# DRAM traffic per launch of the dominant kernel, from one ncu capture, keyed by
-# (workload, kernel) together with the hash of the kernel's source file at the
-# time of the capture; a changed source makes the figure stale (reported null).
-NCU_TRAFFIC = {}
+# DRAM bytes (read + write) per launch of the dominant kernel, from one ncu
+# capture each (profiles/ holds the summaries); a record counts only while its
+# kernel's source file is unchanged (hash of the .cu).
+NCU_TRAFFIC = {
+    ("decode", "decode_gate_up_kernel"): {"bytes": 488557824, "src": "5081ecfb3dbd224e", "from": "profiles/decode_gate_up_kernel__decode.md: full workload"},
+    ("prefill", "grouped_gemm_bf16_kernel<256,true>"): {"bytes": 2480920224, "src": "af7a22686085ba56", "from": "profiles/grouped_gemm_bf16__prefill.md: full workload"},
+    ("fp8", "grouped_gemm_e4m3_kernel<true>"): {"bytes": 10927270336, "src": "02b71bcb1dc5f707", "from": "profiles/grouped_gemm_e4m3__fp8_1024tok_64exp.md: T=1024, E=64 capture x4 (rows and experts scale by 4)"},
+    ("fp8_decode", "decode_e4m3_gate_up_kernel"): {"bytes": 2841453056, "src": "4ecd5f69f521259e", "from": "profiles/decode_e4m3_gate_up_kernel__fp8_2tok_32exp.md: T=2, E=32 capture (14 touched experts) x 94/14 touched"},
+}
 
 
 def log(*a):
