@@ -35,7 +35,8 @@ namespace {
 
 constexpr int kBK = 64;  // bf16 elements per 128-byte row of a stage
 constexpr int kStages = 4;
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;  // producer, MMA issuer, 8 epilogue warps
+constexpr int kEpiWarps = 8;
 
 struct GemmParams {
   const int* mt_base;  // [E+1] per-expert 128-row tile prefix
@@ -80,6 +81,29 @@ struct Layout {
   }
 };
 
+// act(gate) * up for this thread's row: TMEM columns [64*half, 64*half+64) of
+// the gate block and the same of the up block, written as 64 bf16 h values.
+template <int kAct>
+__device__ __forceinline__ void epilogue_gated(uint32_t tb, int half, bool valid, __nv_bfloat16* dst) {
+#pragma unroll 1
+  for (int cc = 2 * half; cc < 2 * half + 2; ++cc) {
+    uint32_t g[32], u[32];
+    tmem_ld32(tb + cc * 32, g);
+    tmem_ld32(tb + 128 + cc * 32, u);
+    tmem_ld_wait();
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      pk[i] = pack_bf16x2(gated_act_t<kAct>(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i])),
+                          gated_act_t<kAct>(__uint_as_float(g[2 * i + 1]), __uint_as_float(u[2 * i + 1])));
+    if (valid) {
+      uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+    }
+  }
+}
+
 template <int kN, bool kSwiGLU>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -109,7 +133,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 4);
+      mbar_init(&tempty[b], kEpiWarps);
     }
     mbar_init(drain, 1);
     *s_abort = 0;
@@ -217,7 +241,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ---------------- epilogue ----------------
-    const int quad = warp & 3;  // TMEM lanes 32*quad .. 32*quad+31 belong to this warp
+    // two warps per TMEM lane quadrant (a warp may only read lanes
+    // 32*(warp%4) .. +31), each converting half of the tile's columns
+    const int quad = warp & 3;
+    const int half = (warp - 2) >> 2;
     const int r = quad * 32 + lane;
     int acc = 0;
     uint32_t aph = 0;
@@ -232,26 +259,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       __nv_bfloat16* dst =
           p.out + static_cast<size_t>(c.row0 + r) * p.out_ld + static_cast<size_t>(c.n) * p.out_tile_cols;
       if constexpr (kSwiGLU) {
-#pragma unroll 1
-        for (int cc = 0; cc < 4; ++cc) {
-          uint32_t g[32], u[32];
-          tmem_ld32(tb + cc * 32, g);
-          tmem_ld32(tb + 128 + cc * 32, u);
-          tmem_ld_wait();
-          uint32_t pk[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i)
-            pk[i] = pack_bf16x2(gated_act(p.act, __uint_as_float(g[2 * i]), __uint_as_float(u[2 * i])),
-                                gated_act(p.act, __uint_as_float(g[2 * i + 1]), __uint_as_float(u[2 * i + 1])));
-          if (valid) {
-            uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-          }
+        // gate columns 0..127, up columns 128..255 of the accumulator
+        switch (p.act) {
+          case MOE_ACT_GELU: epilogue_gated<MOE_ACT_GELU>(tb, half, valid, dst); break;
+          case MOE_ACT_RELU: epilogue_gated<MOE_ACT_RELU>(tb, half, valid, dst); break;
+          default: epilogue_gated<MOE_ACT_SILU>(tb, half, valid, dst); break;
         }
       } else {
+        constexpr int kChunks = kN / 32 / 2;  // 32-column chunks per half
 #pragma unroll 1
-        for (int cc = 0; cc < kN / 32; ++cc) {
+        for (int cc = half * kChunks; cc < (half + 1) * kChunks; ++cc) {
           uint32_t v[32];
           tmem_ld32(tb + cc * 32, v);
           tmem_ld_wait();

@@ -10,6 +10,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "../../include/moe_b200.h"
+
 namespace moe {
 
 // Bits of the device status word (workspace offset `status`).
@@ -308,6 +310,21 @@ __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v 
 // act(g) * u in fp32 for the gated activations (moe_activation):
 // silu(z) = z / (1 + exp(-z)), gelu(z) = z/2 * (1 + erf(z / sqrt 2)), relu(z) = max(z, 0).
 // `act` is uniform across a kernel, so the branch never diverges.
+// The same with the activation fixed at compile time (no branch per element);
+// silu's division uses the fast reciprocal form, whose error (a few ulp of
+// fp32) is far below the bf16 rounding of h.
+template <int kAct>
+__device__ __forceinline__ float gated_act_t(float g, float u) {
+  float a;
+  if (kAct == MOE_ACT_GELU)
+    a = 0.5f * g * (1.0f + erff(g * 0.7071067811865476f));
+  else if (kAct == MOE_ACT_RELU)
+    a = fmaxf(g, 0.0f);
+  else
+    a = __fdividef(g, 1.0f + __expf(-g));
+  return a * u;
+}
+
 __device__ __forceinline__ float gated_act(int act, float g, float u) {
   float a;
   if (act == 1)
