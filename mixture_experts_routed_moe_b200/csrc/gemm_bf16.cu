@@ -16,10 +16,12 @@
 // of many small experts runs in clusters of two CTAs that walk the tiles
 // together, one N block each, so they also share the activation rows.
 //
-// Warp roles (192 threads, one CTA per SM):
+// Warp roles (320 threads, one CTA per SM):
 //   warp 0      TMA producer: A tile [128 x 64] and B tile [N x 64] per stage
 //   warp 1      TMEM allocator and MMA issuer (one thread): 4 MMAs of K=16 per stage
-//   warps 2..5  epilogue: TMEM -> registers -> SwiGLU / bf16 -> global memory
+//   warps 2..9  epilogue: TMEM -> registers -> act(gate)*up / bf16 -> global
+//               memory; two warps per TMEM lane quadrant, half the columns each
+//               (with four, the epilogue took as long as a tile's MMAs)
 // Shared memory holds a 4-stage ring; TMEM holds two accumulators of N fp32
 // columns so the epilogue of one tile overlaps the MMAs of the next.
 // For gate/up, B stacks the 128 gate rows n..n+127 (expert rows n) over the 128
