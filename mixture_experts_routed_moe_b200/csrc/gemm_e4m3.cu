@@ -63,6 +63,41 @@ struct Fp8Params {
 
 __device__ __forceinline__ void epi_bar_sync() { asm volatile("bar.sync 1, %0;" ::"n"(32 * kEpiWarps) : "memory"); }
 
+// End of a gate/up tile for one thread's row: h = act(gate) * up on its 64
+// columns, the row's amax over the 128-column group (this warp's half and the
+// partner warp's, exchanged through shared memory), then the 1x128 e4m3 codes
+// and the group scale. The activation is fixed at compile time.
+template <int kAct>
+__device__ __forceinline__ void finish_gate_up(float (&acc)[128], float* s_amax, int hf, int r, bool valid,
+                                               uint8_t* hrow, float* hs) {
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 64; ++i) {
+    acc[i] = gated_act_t<kAct>(acc[i], acc[64 + i]);
+    amax = fmaxf(amax, fabsf(acc[i]));
+  }
+  s_amax[hf * kTileM + r] = amax;
+  epi_bar_sync();
+  amax = fmaxf(s_amax[r], s_amax[kTileM + r]);
+  epi_bar_sync();
+  const float sc = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+  if (valid) {
+    uint32_t w[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(__fdiv_rn(acc[4 * i], sc), __fdiv_rn(acc[4 * i + 1], sc)),
+                                                   __NV_SATFINITE, __NV_E4M3);
+      const uint32_t hi = __nv_cvt_float2_to_fp8x2(
+          make_float2(__fdiv_rn(acc[4 * i + 2], sc), __fdiv_rn(acc[4 * i + 3], sc)), __NV_SATFINITE, __NV_E4M3);
+      w[i] = lo | (hi << 16);
+    }
+    uint4* dst = reinterpret_cast<uint4*>(hrow);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+    if (hf == 0) *hs = sc;
+  }
+}
+
 template <bool kGateUp>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_e4m3_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -229,15 +264,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t tb = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(pb * 256);
         // gate/up: columns [64hf, 64hf+64) of the gate half and the same of the up half;
         // down: columns [128hf, 128hf+128)
+        // two 16-column loads in flight per wait
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const uint32_t col = kGateUp ? ((q < 4 ? 0u : 128u) + 64u * hf + 16u * (q & 3)) : (128u * hf + 16u * q);
-          uint32_t v[16];
-          tmem_ld16(tb + col, v);
+        for (int q = 0; q < 8; q += 2) {
+          uint32_t v[2][16];
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const int qq = q + j;
+            const uint32_t col =
+                kGateUp ? ((qq < 4 ? 0u : 128u) + 64u * hf + 16u * (qq & 3)) : (128u * hf + 16u * qq);
+            tmem_ld16(tb + col, v[j]);
+          }
           tmem_ld_wait();
-          const float sc = (kGateUp && q >= 4) ? sc1 : sc0;
 #pragma unroll
-          for (int i = 0; i < 16; ++i) acc[16 * q + i] = fmaf(__uint_as_float(v[i]), sc, acc[16 * q + i]);
+          for (int j = 0; j < 2; ++j) {
+            const int qq = q + j;
+            const float sc = (kGateUp && qq >= 4) ? sc1 : sc0;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) acc[16 * qq + i] = fmaf(__uint_as_float(v[j][i]), sc, acc[16 * qq + i]);
+          }
         }
         tc_fence_before();
         __syncwarp();
@@ -252,31 +297,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool valid = r < c.valid;
       if constexpr (kGateUp) {
         // h for columns n*128 + 64hf + i, i < 64: acc[i] is the gate, acc[64+i] the up projection
-        float amax = 0.f;
-#pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          acc[i] = gated_act(p.act, acc[i], acc[64 + i]);
-          amax = fmaxf(amax, fabsf(acc[i]));
-        }
-        s_amax[hf * kTileM + r] = amax;
-        epi_bar_sync();
-        amax = fmaxf(s_amax[r], s_amax[kTileM + r]);
-        epi_bar_sync();
-        const float sc = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
-        if (valid) {
-          uint32_t w[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const uint32_t lo = __nv_cvt_float2_to_fp8x2(
-                make_float2(__fdiv_rn(acc[4 * i], sc), __fdiv_rn(acc[4 * i + 1], sc)), __NV_SATFINITE, __NV_E4M3);
-            const uint32_t hi = __nv_cvt_float2_to_fp8x2(
-                make_float2(__fdiv_rn(acc[4 * i + 2], sc), __fdiv_rn(acc[4 * i + 3], sc)), __NV_SATFINITE, __NV_E4M3);
-            w[i] = lo | (hi << 16);
-          }
-          uint4* dst = reinterpret_cast<uint4*>(p.hq + static_cast<size_t>(row) * p.out_ld + c.n * 128 + hf * 64);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
-          if (hf == 0) p.hs[static_cast<size_t>(row) * (p.out_ld / 128) + c.n] = sc;
+        uint8_t* hrow = p.hq + static_cast<size_t>(row) * p.out_ld + c.n * 128 + hf * 64;
+        float* hs = p.hs + static_cast<size_t>(row) * (p.out_ld / 128) + c.n;
+        switch (p.act) {
+          case MOE_ACT_GELU: finish_gate_up<MOE_ACT_GELU>(acc, s_amax, hf, r, valid, hrow, hs); break;
+          case MOE_ACT_RELU: finish_gate_up<MOE_ACT_RELU>(acc, s_amax, hf, r, valid, hrow, hs); break;
+          default: finish_gate_up<MOE_ACT_SILU>(acc, s_amax, hf, r, valid, hrow, hs); break;
         }
       } else {
         if (valid) {
