@@ -113,10 +113,17 @@ __device__ __forceinline__ void scan_experts(int* __restrict__ counts, int nblk,
   const int e = threadIdx.x;
   int c = 0;
   if (e < E) {
-    for (int b = 0; b < nblk; ++b) {
-      const int v = counts[static_cast<size_t>(b) * E + e];
-      counts[static_cast<size_t>(b) * E + e] = c;
-      c += v;
+    // exclusive prefix over the blocks, eight independent loads in flight at a
+    // time (one dependent load per block made this a chain of global latencies)
+    for (int b0 = 0; b0 < nblk; b0 += 8) {
+      int v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = b0 + j < nblk ? counts[static_cast<size_t>(b0 + j) * E + e] : 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (b0 + j < nblk) counts[static_cast<size_t>(b0 + j) * E + e] = c;
+        c += v[j];
+      }
     }
     cnt[e] = c;
   }
