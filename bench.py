@@ -332,6 +332,53 @@ def stage_roofline(wl, path, stage_ms, n_touched, peaks, peak_src):
     return out
 
 
+def time_router(moe, wl, seed, xd, flush, stream, K, W, world, peaks):
+    """The fused router (moe_router: x W_r^T and the top-k routing in one
+    kernel) on the workload's tokens, with router weights ~ N(0, 0.02): its own
+    CUDA-event time per launch, L2 flushed between launches, and its roofline
+    (algorithmic bytes x + W_r + routing outputs; FLOPs 2*T*H*E)."""
+    w_r = G.make_router_weights(wl, seed, device=xd.device)
+    # one launch captured in a CUDA graph, so the events time the kernel and
+    # not the host's call overhead
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        for _ in range(max(W, 1)):
+            moe.router(xd, w_r, wl.k)
+    stream.wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        moe.router(xd, w_r, wl.k)
+    for _ in range(W):
+        g.replay()
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    torch.cuda.synchronize()
+    for i in range(K):
+        flush.zero_()
+        ev_s[i].record(stream)
+        g.replay()
+        ev_e[i].record(stream)
+    torch.cuda.synchronize()
+    del g
+    ms = max_over_ranks(sum(ev_s[i].elapsed_time(ev_e[i]) for i in range(K)), world) / K
+    flops = 2 * wl.T * wl.H * wl.E
+    byts = wl.T * wl.H * 2 + wl.E * wl.H * 2 + wl.T * wl.k * 8
+    t_tensor = flops / (peaks["bf16_tflops"] * 1e12)
+    t_hbm = byts / (peaks["hbm_gbs"] * 1e9)
+    if t_tensor >= t_hbm:
+        ach = flops / (ms / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": ach / peaks["bf16_tflops"]}
+    else:
+        ach = byts / (ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": ach / peaks["hbm_gbs"]}
+    roof.update({"kernel": "router_kernel", "algorithmic_flops": flops, "algorithmic_bytes": byts})
+    return {"ms": ms, "tokens_per_s": wl.T / (ms / 1e3), "launches": K, "roofline": roof}
+
+
 def run_ours(args, world, rank, local):
     import mixture_experts_routed_moe_b200 as moe
 
@@ -417,6 +464,10 @@ def run_ours(args, world, rank, local):
         raise RuntimeError("graph replay and eager forward disagree")
 
     peaks, peak_src = load_peaks()
+    router_line = None
+    if args.router and wl.E <= 256:
+        router_line = time_router(moe, wl, seed, xd, flush, stream, K, args.warmup, world, peaks)
+
     # route, permute, gate/up, down, combine; the e4m3 DECODE path adds the
     # per-token x quantisation and the h quantisation
     per_step_launches = (1 + (1 if wl.T <= 256 else 3) + 2 + 1
@@ -438,6 +489,8 @@ def run_ours(args, world, rank, local):
         "gpu_launches": per_step_launches * K,
         "clocks": clk,
     }
+    if router_line is not None:
+        line["router"] = router_line
     # stage indices above: events[0..4] = before permute, after permute, after gate/up, after down, after combine
     line["roofline"] = stage_roofline(wl, path, {1: stage_ms[2], 2: stage_ms[3]}, n_touched, peaks, peak_src)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -457,6 +510,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=list(G.WORKLOADS), default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--router", action="store_true",
+                    help="also time the fused router (router GEMM + top-k) on the workload's tokens")
     ap.add_argument("--shape", default=None,
                     help="T,H,I,E,k,wdtype: a custom layer instead of a named workload (profiling-sized cases)")
     args = ap.parse_args()

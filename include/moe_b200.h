@@ -76,8 +76,8 @@ typedef struct {
 } moe_shape;
 
 /*
- * moe_route -- router top-k ("Experts backends", introduction: "a router
- * selects k experts"). For each token t: softmax over the E fp32 logits, the k
+ * moe_route -- router top-k ("Experts backends", introduction: the router
+ * picks k experts per token). For each token t: softmax over the E fp32 logits, the k
  * experts with the largest logits (equal logits: lower index first), slot j
  * holding the j-th largest, and their probabilities renormalised to sum to 1.
  *
@@ -88,6 +88,29 @@ typedef struct {
  */
 moe_status moe_route(const float* logits, int32_t T, int32_t E, int32_t k,
                      int32_t* topk_idx, float* topk_w, void* stream);
+
+/*
+ * moe_router -- the router GEMM fused with moe_route (the step ahead of the
+ * experts: "Experts backends", introduction, the router that picks k experts;
+ * backend table, row "sonicmoe", which fuses the router dispatch with the
+ * expert GEMMs). For each token t:
+ *   logits[t, e] = sum_h x[t, h] * w_router[e, h]   (bf16 inputs, fp32 accumulation)
+ * then exactly moe_route's selection and weights on those fp32 logits (the
+ * same code: for equal logits both give the same bits).
+ *
+ *   x          [T, H] bf16, 16-byte aligned
+ *   w_router   [E, H] bf16, 16-byte aligned
+ *   logits     [T, E] fp32 out, or NULL when the logits are not wanted
+ *   topk_idx   [T, k] int32 out
+ *   topk_w     [T, k] fp32 out
+ * Requirements: T >= 0; H a positive multiple of 64 (at most 65536);
+ * 1 <= k <= E <= 256. T == 0 is a no-op. Errors: MOE_ERR_INVALID_ARG before
+ * any launch; MOE_ERR_CUDA for a failed launch. A bounded device wait that
+ * gives up (never in normal operation) writes topk_idx = -1 for the tokens of
+ * the affected 128-token tile.
+ */
+moe_status moe_router(const void* x, const void* w_router, int32_t T, int32_t H, int32_t E, int32_t k,
+                      float* logits, int32_t* topk_idx, float* topk_w, void* stream);
 
 /* Bytes of device workspace moe_forward needs for `shape` (an upper bound
  * that depends only on the shape; host-only, enqueues nothing). Returns 0 for

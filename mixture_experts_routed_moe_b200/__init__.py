@@ -29,7 +29,7 @@ ACT = {"silu": 0, "gelu": 1, "relu": 2}
 PATH_NAMES = {v: k for k, v in PATH.items()}
 EXPORTS = ["moe_route", "moe_workspace_size", "moe_forward", "moe_forward_timed", "moe_workspace_query",
            "moe_read_device_status", "moe_status_string", "moe_version", "moe_forward_noalloc",
-           "moe_set_test_hooks"]
+           "moe_set_test_hooks", "moe_router"]
 
 
 class MoeError(RuntimeError):
@@ -78,6 +78,8 @@ def lib() -> ctypes.CDLL:
         L.moe_status_string.restype = ctypes.c_char_p
         L.moe_forward_noalloc.argtypes = [ctypes.POINTER(MoeShape), vp, vp, vp, vp, vp, vp, vp, vp, vp]
         L.moe_forward_noalloc.restype = i32
+        L.moe_router.argtypes = [vp, vp, i32, i32, i32, i32, vp, vp, vp, vp]
+        L.moe_router.restype = i32
         L.moe_set_test_hooks.argtypes = [i32, ctypes.c_uint64]
         L.moe_set_test_hooks.restype = i32
         L.moe_version.argtypes = []
@@ -192,6 +194,21 @@ def read_device_status(workspace: torch.Tensor, stream=None) -> int:
     return int(lib().moe_read_device_status(_ptr(workspace), _stream(stream)))
 
 
+def router(x: torch.Tensor, w_router: torch.Tensor, k: int, logits: bool = False, stream=None):
+    """moe_router: logits = x w_router^T (bf16 in, fp32 accumulate) and the
+    top-k routing on them, in one kernel. x bf16 [T,H], w_router bf16 [E,H].
+    Returns (topk_idx int32 [T,k], topk_w fp32 [T,k]) and, with logits=True,
+    the fp32 logits [T,E] as a third element."""
+    T, H = x.shape
+    E = w_router.shape[0]
+    idx = torch.empty((T, k), dtype=torch.int32, device=x.device)
+    w = torch.empty((T, k), dtype=torch.float32, device=x.device)
+    lg = torch.empty((T, E), dtype=torch.float32, device=x.device) if logits else None
+    _check(lib().moe_router(_ptr(x), _ptr(w_router), T, H, E, k, _ptr(lg), _ptr(idx), _ptr(w), _stream(stream)),
+           "moe_router")
+    return (idx, w, lg) if logits else (idx, w)
+
+
 def set_test_hooks(stall_gate_up_loads: bool = False, wait_limit_ns: int = 0) -> None:
     """Failure-detection test switches (moe_set_test_hooks): the limit of every
     bounded device wait (0 = the 2 s default) and a stall of the prefill
@@ -264,5 +281,5 @@ class MoEGraph:
 
 
 __all__ = ["lib", "route", "forward", "forward_noalloc", "MoEGraph", "workspace_size", "workspace_layout", "alloc_workspace",
-           "read_device_status", "set_test_hooks", "make_shape", "MoELayer", "MoeError", "MoeShape", "EXPORTS", "STATUS",
+           "read_device_status", "set_test_hooks", "router", "make_shape", "MoELayer", "MoeError", "MoeShape", "EXPORTS", "STATUS",
            "status_string", "PATH", "WDTYPE", "ACT"]

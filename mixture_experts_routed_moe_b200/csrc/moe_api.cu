@@ -287,6 +287,22 @@ moe_status moe_workspace_query(const moe_shape* shape, moe_workspace_layout* lay
   return MOE_OK;
 }
 
+moe_status moe_router(const void* x, const void* w_router, int32_t T, int32_t H, int32_t E, int32_t k,
+                      float* logits, int32_t* topk_idx, float* topk_w, void* stream) {
+  if (T < 0 || H < 64 || H % 64 != 0 || H > 65536 || E < 1 || E > 256 || k < 1 || k > E) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (x == nullptr || w_router == nullptr || topk_idx == nullptr || topk_w == nullptr) return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(w_router, 16) || !aligned(topk_idx, 4) || !aligned(topk_w, 4) ||
+      !aligned(logits, 4))
+    return MOE_ERR_INVALID_ARG;
+  if (static_cast<long long>(T) * k >= (1ll << 31) || static_cast<long long>(T) * E >= (1ll << 40))
+    return MOE_ERR_INVALID_ARG;
+  return launch_router(x, w_router, T, H, E, k, logits, topk_idx, topk_w, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
+}
+
 moe_status moe_set_test_hooks(int32_t stall_gate_up_loads, uint64_t wait_limit_ns) {
   if (stall_gate_up_loads != 0 && stall_gate_up_loads != 1) return MOE_ERR_INVALID_ARG;
   if (wait_limit_ns != 0 && (wait_limit_ns < 1000000ull || wait_limit_ns > 60000000000ull)) return MOE_ERR_INVALID_ARG;

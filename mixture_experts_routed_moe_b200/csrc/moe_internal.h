@@ -42,6 +42,10 @@ bool make_plan(const moe_shape* s, Plan* p);
 // Launchers. Each returns the launch's cudaError_t.
 cudaError_t launch_route(const float* logits, int T, int E, int k, int* idx, float* w, cudaStream_t st);
 
+// Router GEMM + routing (E <= 256, H % 64 == 0); logits may be null.
+cudaError_t launch_router(const void* x, const void* w_router, int T, int H, int E, int k, float* logits, int* idx,
+                          float* w, cudaStream_t st);
+
 cudaError_t launch_permute(const moe_shape* s, const Plan& p, const int* topk_idx, const void* x, uint8_t* ws,
                            cudaStream_t st);
 

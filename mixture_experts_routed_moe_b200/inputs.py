@@ -166,6 +166,15 @@ def make_expert_weights(wl: Workload, seed: int, e: int, device="cpu"):
     return dict(w_gate_up=qa, w_down=qb, sw_gate_up=sa, sw_down=sb)
 
 
+def make_router_weights(wl: Workload, seed: int, device="cpu") -> torch.Tensor:
+    """Router weights W_r [E, H] ~ N(0, 0.02) as bf16, from a torch generator
+    on `device` (seed * 100003 + 99991, apart from every expert's stream)."""
+    g = torch.Generator(device=device)
+    g.manual_seed(seed * 100003 + 99991)
+    w = torch.randn((wl.E, wl.H), generator=g, device=device, dtype=torch.float32) * 0.02
+    return w.to(torch.bfloat16)
+
+
 def routed_inputs_with_counts(wl: Workload, counts, seed: int = 0):
     """Hand-placed routing for edge cases: a [T,k] int32 choice in which expert e
     is picked by exactly counts[e] tokens (sum(counts) == T*k, max(counts) <= T),
@@ -211,6 +220,7 @@ def ceil_div(a: int, b: int) -> int:
 
 __all__ = [
     "Workload", "WORKLOADS", "WORKLOAD_ORDER", "default_seed", "make_activations", "make_weights",
-    "make_expert_weights", "quantize_weight_blocks", "routed_inputs_with_counts", "flops_and_bytes",
+    "make_expert_weights", "make_router_weights", "quantize_weight_blocks", "routed_inputs_with_counts",
+    "flops_and_bytes",
     "router_bias", "ceil_div",
 ]

@@ -135,9 +135,10 @@ def ue8m0_scale(b) -> np.ndarray:
 def route(logits, k: int):
     """Top-k routing of fp32 router logits [T, E].
 
-    Experts backends, introduction ("a router selects k experts ... aggregated
-    with the routing weights"). Softmax over all experts, choose the k largest
-    (R1), renormalise their probabilities over the k (R2).
+    Experts backends, introduction: the router picks k experts per token and
+    their outputs are summed with the routing weights. Softmax over all
+    experts, choose the k largest (R1), renormalise their probabilities over
+    the k (R2).
 
     Returns (topk_idx int32 [T,k], topk_w float32 [T,k], topk_w64 float64 [T,k])."""
     L = np.asarray(logits, dtype=np.float32).astype(np.float64)
@@ -153,6 +154,15 @@ def route(logits, k: int):
     sel = np.take_along_axis(p, idx.astype(np.int64), axis=1)
     w64 = sel / sel.sum(axis=1, keepdims=True)
     return idx, w64.astype(np.float32), w64
+
+
+def router_logits(x, w_router):
+    """Router logits [T, E] = x W_r^T, float64, from the given (bf16-valued)
+    x [T, H] and router weights W_r [E, H]: the router step ahead of the experts
+    (backend table, row "sonicmoe", which fuses the router dispatch with the
+    expert GEMMs; the introduction's router that picks k experts per token).
+    The routing itself is route() on these logits."""
+    return np.asarray(x, dtype=np.float64) @ np.asarray(w_router, dtype=np.float64).T
 
 
 # ---------------------------------------------------------------------------

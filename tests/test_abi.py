@@ -117,6 +117,16 @@ def test_route_host_errors(L):
     assert L.moe_route(None, 0, 8, 2, None, None, None) == 0
 
 
+def test_router_host_errors(L):
+    # (x, w_router, T, H, E, k, logits, idx, w, stream)
+    assert L.moe_router(FAKE, FAKE, 4, 128, 257, 2, None, FAKE, FAKE, None) == -1  # E > 256
+    assert L.moe_router(FAKE, FAKE, 4, 100, 8, 2, None, FAKE, FAKE, None) == -1  # H not a multiple of 64
+    assert L.moe_router(FAKE, FAKE, 4, 128, 8, 9, None, FAKE, FAKE, None) == -1  # k > E
+    assert L.moe_router(FAKE + 8, FAKE, 4, 128, 8, 2, None, FAKE, FAKE, None) == -1  # misaligned x
+    assert L.moe_router(None, FAKE, 4, 128, 8, 2, None, FAKE, FAKE, None) == -1
+    assert L.moe_router(None, None, 0, 128, 8, 2, None, None, None, None) == 0  # T == 0: nothing to do
+
+
 def test_test_hooks_validate_and_reset(L):
     assert L.moe_set_test_hooks(2, 0) == -1
     assert L.moe_set_test_hooks(0, 999_999) == -1  # below 1 ms

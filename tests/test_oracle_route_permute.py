@@ -109,3 +109,35 @@ def test_permute_invariants_and_brute_force(T, E, k, BM):
         assert (blk[:cnt[e]] >= 0).all() and (blk[cnt[e]:] == -1).all()
         assert (idx.ravel()[blk[:cnt[e]]] == e).all()
         assert (np.diff(blk[:cnt[e]] // k) > 0).all()  # ascending tokens
+
+
+# ---------------------------------------------------------------------------
+# router logits (the router GEMM ahead of the routing)
+# ---------------------------------------------------------------------------
+
+def test_router_logits_one_hot_rows_select_weight_columns():
+    rng = np.random.default_rng(7)
+    E, H = 5, 12
+    w = rng.standard_normal((E, H))
+    x = np.zeros((H, H))
+    x[np.arange(H), np.arange(H)] = 1.0  # token h is the unit vector e_h
+    np.testing.assert_array_equal(O.router_logits(x, w), w.T)
+
+
+def test_router_logits_brute_force_and_linearity():
+    rng = np.random.default_rng(8)
+    T, E, H = 4, 3, 6
+    x = rng.standard_normal((T, H))
+    w = rng.standard_normal((E, H))
+    L = O.router_logits(x, w)
+    for t in range(T):
+        for e in range(E):
+            s = 0.0
+            for h in range(H):
+                s += x[t, h] * w[e, h]
+            assert abs(L[t, e] - s) < 1e-12
+    x2 = rng.standard_normal((T, H))
+    np.testing.assert_allclose(O.router_logits(2.0 * x - 3.0 * x2, w), 2.0 * L - 3.0 * O.router_logits(x2, w),
+                               rtol=1e-12, atol=1e-12)
+    # a transposed weight matrix cannot be applied, and swapped operands give E x T
+    assert O.router_logits(x, w).shape == (T, E)
