@@ -310,6 +310,11 @@ cudaError_t launch_one(const CUtensorMap& tmA, const CUtensorMap& tmB, const Gem
     grouped_gemm_bf16_kernel<kN, kSwiGLU><<<grid, kThreads, smem, st>>>(tmA, tmB, gp);
     return cudaGetLastError();
   }
+  // every cluster of the persistent grid must be resident at once: with an
+  // odd SM count in a GPC, fewer than num_sms / cs clusters fit
+  const int maxc = max_active_clusters(reinterpret_cast<const void*>(grouped_gemm_bf16_kernel<kN, kSwiGLU>), gp.cs,
+                                       kThreads, smem);
+  if (maxc > 0) grid = std::min(grid, gp.cs * maxc);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);  // a multiple of gp.cs
   cfg.blockDim = dim3(kThreads, 1, 1);

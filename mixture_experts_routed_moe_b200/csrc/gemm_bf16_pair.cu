@@ -254,6 +254,11 @@ cudaError_t launch_pair(const CUtensorMap& tmA, const CUtensorMap& tmB, const Pa
   static unsigned long long done = 0;
   cudaError_t err = ensure_max_smem(reinterpret_cast<const void*>(grouped_gemm_bf16_pair_kernel), &done);
   if (err != cudaSuccess) return err;
+  // every pair of the persistent grid must be resident at once: with an odd
+  // SM count in a GPC, fewer than num_sms / 2 pairs fit
+  const int maxc = max_active_clusters(reinterpret_cast<const void*>(grouped_gemm_bf16_pair_kernel), 2, kThreads,
+                                       pair_smem_bytes(pp.E));
+  if (maxc > 0) nclusters = std::min(nclusters, maxc);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * nclusters, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);

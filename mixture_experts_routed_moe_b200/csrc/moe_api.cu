@@ -6,6 +6,8 @@
 #include <atomic>
 #include <cstring>
 #include <limits>
+#include <mutex>
+#include <vector>
 
 #include "moe_common.cuh"
 #include "moe_internal.h"
@@ -153,6 +155,41 @@ bool make_plan(const moe_shape* s, Plan* p) {
   p->y = take(M * H * 2);
   p->total = off;
   return true;
+}
+
+int max_active_clusters(const void* kernel, int cluster, int threads, size_t smem) {
+  struct Entry {
+    const void* kernel;
+    int cluster, threads, dev;
+    size_t smem;
+    int n;
+  };
+  static std::mutex mu;
+  static std::vector<Entry> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  std::lock_guard<std::mutex> lock(mu);
+  for (const Entry& e : cache)
+    if (e.kernel == kernel && e.cluster == cluster && e.threads == threads && e.dev == dev && e.smem == smem)
+      return e.n;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(cluster), 1, 1);
+  cfg.blockDim = dim3(static_cast<unsigned>(threads), 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(cluster);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess) {
+    cudaGetLastError();  // clear the query's error; callers fall back to their own bound
+    n = 0;
+  }
+  cache.push_back(Entry{kernel, cluster, threads, dev, smem, n});
+  return n;
 }
 
 unsigned long long wait_limit_ns() { return g_wait_limit_ns.load(std::memory_order_relaxed); }

@@ -85,4 +85,10 @@ int device_sm_count();
 // captured in CUDA graphs). `done` is one bitmask per kernel, bit = device.
 cudaError_t ensure_max_smem(const void* kernel, unsigned long long* done);
 
+// Clusters of `cluster` CTAs (each `threads` threads and `smem` bytes of
+// dynamic shared memory) of `kernel` that the current device holds at once;
+// cached per kernel, shape and device; 0 if the query fails. A persistent
+// cluster grid larger than this leaves clusters waiting for a second wave.
+int max_active_clusters(const void* kernel, int cluster, int threads, size_t smem);
+
 }  // namespace moe
