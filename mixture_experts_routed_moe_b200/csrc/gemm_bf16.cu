@@ -389,13 +389,7 @@ cudaError_t launch_gemm_bf16(const moe_shape* s, const Plan& p, const void* w_ga
   gp.b_second_offset = 128;
   gp.out = reinterpret_cast<__nv_bfloat16*>(ws + p.y);
   gp.out_ld = H;
-  if (H % 256 == 0) {
-    gp.n_tiles = H / 256;
-    gp.b_tile_stride = 256;
-    gp.out_tile_cols = 256;
-    const int grid = std::max(1, std::min(num_sms, max_mtiles * gp.n_tiles));
-    return launch_one<256, false>(tmA, tmB, gp, grid, st);
-  }
+  // (H % 256 == 0 runs on the CTA-pair kernel, gemm_bf16_pair.cu)
   gp.n_tiles = H / 128;
   gp.b_tile_stride = 128;
   gp.out_tile_cols = 128;

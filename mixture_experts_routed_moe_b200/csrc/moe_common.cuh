@@ -102,15 +102,6 @@ __device__ __forceinline__ void tma_load_2d_hint(void* smem_dst, const CUtensorM
       : "memory");
 }
 
-// Plain bulk copy of `bytes` (multiple of 16, both addresses 16-byte aligned)
-// from global to shared memory, completing on `bar` with complete_tx.
-__device__ __forceinline__ void bulk_copy_g2s(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                   smem_u32(smem_dst)),
-               "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
-               : "memory");
-}
-
 // L2 cache policies for TMA loads.
 __device__ __forceinline__ uint64_t l2_policy_evict_last() {
   uint64_t pol;
@@ -361,18 +352,6 @@ __device__ __forceinline__ uint4 ld_stream_u4(const void* p) {
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                : "l"(p));
   return v;
-}
-
-__device__ __forceinline__ float dot8_bf16(const uint4& a, const uint4& b, float acc) {
-  acc = fmaf(bf16_lo(a.x), bf16_lo(b.x), acc);
-  acc = fmaf(bf16_hi(a.x), bf16_hi(b.x), acc);
-  acc = fmaf(bf16_lo(a.y), bf16_lo(b.y), acc);
-  acc = fmaf(bf16_hi(a.y), bf16_hi(b.y), acc);
-  acc = fmaf(bf16_lo(a.z), bf16_lo(b.z), acc);
-  acc = fmaf(bf16_hi(a.z), bf16_hi(b.z), acc);
-  acc = fmaf(bf16_lo(a.w), bf16_lo(b.w), acc);
-  acc = fmaf(bf16_hi(a.w), bf16_hi(b.w), acc);
-  return acc;
 }
 
 }  // namespace moe
