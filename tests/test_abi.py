@@ -74,6 +74,23 @@ def test_workspace_layout_is_consistent(L):
         assert (lay.xa == 2 ** 64 - 1) == (path == "decode")
 
 
+def test_e4m3_workspace_layouts(L):
+    """e4m3 PREFILL: x codes per permuted row; e4m3 DECODE: x codes once per
+    token (T rows), then h codes and scales per assignment row."""
+    T, H, I, E, k = 16, 7168, 2048, 256, 8
+    pre = moe.workspace_layout(shape(T=T, H=H, I=I, E=E, k=k, wdtype="e4m3", path="prefill"))
+    dec = moe.workspace_layout(shape(T=T, H=H, I=I, E=E, k=k, wdtype="e4m3", path="decode"))
+    assert dec.bm == 1 and dec.m_rows == T * k and pre.bm == 128
+    # decode: xa holds T rows of H codes, xs T rows of H/128 fp32 scales
+    assert dec.xs - dec.xa >= T * H and dec.xs - dec.xa < T * H + 1024
+    assert dec.h - dec.xs >= T * (H // 128) * 4
+    # prefill: one row of codes per permuted row
+    assert pre.xs - pre.xa >= pre.m_rows * H
+    for lay in (pre, dec):
+        assert lay.hs - lay.h >= lay.m_rows * I  # e4m3 h codes
+        assert lay.y + lay.m_rows * H * 2 <= lay.total
+
+
 def test_auto_path_choice(L):
     assert moe.workspace_layout(shape(T=16, H=2048, I=1408, E=60, k=4)).path == moe.PATH["decode"]
     assert moe.workspace_layout(shape(T=8192, H=2048, I=768, E=128, k=8)).path == moe.PATH["prefill"]
