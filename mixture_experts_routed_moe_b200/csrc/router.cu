@@ -26,7 +26,8 @@ namespace moe {
 namespace {
 
 constexpr int kBK = 64;       // K elements per stage (128 bytes of bf16: one swizzle row)
-constexpr int kStages = 4;
+constexpr int kMaxStages = 8;
+constexpr size_t kRingBytes = 192 * 1024;  // shared memory for the TMA ring
 constexpr int kThreads = 192;
 constexpr int kRows = 128;    // tokens per CTA (MMA M)
 constexpr int kA = kRows * kBK * 2;  // 16 KB
@@ -41,9 +42,17 @@ struct RouterParams {
   unsigned long long timeout_ns;
 };
 
+// As many stages as fit the ring (the kernel is bound by the bytes one CTA
+// keeps in flight): 6 for E <= 128, 8 for E <= 64, 4 for E = 256.
+__host__ __device__ constexpr int router_stages(int n_pad) {
+  return static_cast<int>(kRingBytes / static_cast<size_t>(kA + n_pad * kBK * 2)) < kMaxStages
+             ? static_cast<int>(kRingBytes / static_cast<size_t>(kA + n_pad * kBK * 2))
+             : kMaxStages;
+}
+
 __host__ __device__ constexpr size_t router_smem_bytes(int n_pad) {
-  return 1024 /*alignment slack*/ + static_cast<size_t>(kStages) * (kA + n_pad * kBK * 2) + (2 * kStages + 1) * 8 +
-         16;
+  return 1024 /*alignment slack*/ + static_cast<size_t>(router_stages(n_pad)) * (kA + n_pad * kBK * 2) +
+         (2 * kMaxStages + 1) * 8 + 16;
 }
 
 template <int kPerLane>
@@ -53,6 +62,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int kB = p.n_pad * kBK * 2;
+  const int kStages = router_stages(p.n_pad);
   uint8_t* sA = smem;
   uint8_t* sB = smem + kStages * kA;
   uint64_t* full = reinterpret_cast<uint64_t*>(sB + kStages * kB);
