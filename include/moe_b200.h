@@ -3,9 +3,9 @@
  * NVIDIA B200 (sm_100a).
  *
  * The operation (Hugging Face Transformers docs page "Experts backends",
- * introduction): for each token a router selects k experts; the token's hidden
- * state is projected through each selected expert's parameters and the expert
- * outputs are aggregated with the routing weights. Each expert is a gated MLP
+ * introduction): a router chooses k experts per token, each chosen expert maps
+ * the token's hidden state through its own weights, and the token's output is
+ * the routing-weighted sum of those expert results. Each expert is a gated MLP
  * (backend table, row "deepgemm_megamoe"): up projection, SwiGLU, down
  * projection, with SwiGLU meaning silu(gate) * up (section "SonicMoE").
  *

@@ -1,5 +1,6 @@
-// Weighted combine back to token order ("Experts backends", introduction:
-// the expert outputs are aggregated with the routing weights).
+// Weighted combine back to token order ("Experts backends", introduction: a
+// token's result is the sum of its k experts' results, each scaled by the
+// routing weight of that expert).
 //
 //   out[t, :] = bf16( sum_{j = 0..k-1} topk_w[t, j] * y[slot_row[t*k+j], :] )
 //

@@ -1,5 +1,5 @@
-// Router top-k ("Experts backends", introduction: a router selects k experts
-// for each token; the expert outputs are later aggregated with the routing
+// Router top-k ("Experts backends", introduction: each token goes to k experts
+// that a router picks; the experts' results are later summed with the routing
 // weights).
 //
 // One warp per token over logits in global memory; the per-token selection

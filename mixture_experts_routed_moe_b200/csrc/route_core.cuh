@@ -1,6 +1,6 @@
-// Top-k routing of one token by one warp ("Experts backends", introduction: a
-// router selects k experts for each token; the expert outputs are later
-// aggregated with the routing weights). Shared by the routing kernel (logits
+// Top-k routing of one token by one warp ("Experts backends", introduction:
+// each token goes to k experts that a router picks, and the experts' results
+// are later summed with the routing weights). Shared by the routing kernel (logits
 // in global memory) and the fused router GEMM (logits in shared memory), so
 // both give the same bits for the same logits.
 //

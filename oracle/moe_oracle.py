@@ -7,11 +7,11 @@ It shares no code with the CUDA library (no kernels, headers, tables or
 helpers) and imports nothing from it.
 
 Source: Hugging Face Transformers docs page "Experts backends"
-(experts_interface). Its introduction states the computation every backend
-performs: for each token a router picks k experts, the token's hidden state is
-projected through each selected expert's parameters, and the expert outputs are
-aggregated with the routing weights; the backends differ only in how the expert
-matmuls run. The "eager" row of the backend table is the reference
+(experts_interface). Its introduction describes the one computation that all
+backends share: a router chooses k experts per token, every chosen expert maps
+the token's hidden state through its own weights, and the token's output is
+the routing-weighted sum of those expert results; only the way the expert
+matmuls are executed differs between backends. The "eager" row of the backend table is the reference
 implementation: a loop over the selected experts that applies the projections
 to their tokens. That eager loop is the algorithm written out here. The expert
 is a gated MLP: up projection, SwiGLU, down projection (backend table, row
@@ -270,7 +270,7 @@ def _expert_loop(x, topk_idx, E, tokens, mlp):
 
 
 def combine(Y, topk_w, intermediate: str = "bf16"):
-    """out[t] = sum_j w[t,j] * Y[t,j] (introduction: aggregated with the routing weights)."""
+    """out[t] = sum_j w[t,j] * Y[t,j] (introduction: the routing-weighted sum of the experts' results)."""
     w = np.asarray(topk_w, dtype=np.float32).astype(np.float64)
     out = np.zeros((Y.shape[0], Y.shape[2]), dtype=np.float64)
     for j in range(Y.shape[1]):
