@@ -14,7 +14,8 @@ the routing-weighted sum of those expert results; only the way the expert
 matmuls are executed differs between backends. The "eager" row of the backend table is the reference
 implementation: a loop over the selected experts that applies the projections
 to their tokens. That eager loop is the algorithm written out here. The expert
-is a gated MLP: up projection, SwiGLU, down projection (backend table, row
+is a gated MLP: a joint gate/up
+projection, the SwiGLU activation, then the down projection (backend table, row
 "deepgemm_megamoe"; section "Fused Mega MoE on Blackwell"), and the section
 "SonicMoE" maps the gated activations SwiGLU/GeGLU/ReGLU to silu/gelu/relu;
 all three are supported (gelu in its exact erf form).
