@@ -9,16 +9,16 @@ helpers) and imports nothing from it.
 Source: Hugging Face Transformers docs page "Experts backends"
 (experts_interface). Its introduction describes the one computation that all
 backends share: a router chooses k experts per token, every chosen expert maps
-the token's hidden state through its own weights, and the token's output is
-the routing-weighted sum of those expert results; only the way the expert
-matmuls are executed differs between backends. The "eager" row of the backend table is the reference
-implementation: a loop over the selected experts that applies the projections
-to their tokens. That eager loop is the algorithm written out here. The expert
-is a gated MLP: a joint gate/up
-projection, the SwiGLU activation, then the down projection (backend table, row
-"deepgemm_megamoe"; section "Fused Mega MoE on Blackwell"), and the section
-"SonicMoE" maps the gated activations SwiGLU/GeGLU/ReGLU to silu/gelu/relu;
-all three are supported (gelu in its exact erf form).
+the token's hidden state through its own weights, and the token's output is the
+routing-weighted sum of those expert results; only the way the expert matmuls
+are executed differs between backends. The "eager" row of the backend table is
+the reference implementation: a loop over the selected experts that applies the
+projections to their tokens. That eager loop is the algorithm written out here.
+The expert is a gated MLP: a joint gate/up projection, the SwiGLU activation,
+then the down projection (backend table, row "deepgemm_megamoe"; section "Fused
+Mega MoE on Blackwell"), and the section "SonicMoE" maps the gated activations
+SwiGLU/GeGLU/ReGLU to silu/gelu/relu; all three are supported (gelu in its
+exact erf form).
 
 Arithmetic is float64 throughout. The pages fix no precision; where they are
 silent this module takes the readings below (each one is also listed in the
