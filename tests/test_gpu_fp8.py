@@ -160,3 +160,19 @@ def test_fp8_gated_activations(act, path):
                             ExpertView(W["sw_gate_up"], True), ExpertView(W["w_down"], True),
                             ExpertView(W["sw_down"], True), act=act)
     assert assert_fp8_close(out.float().cpu().numpy(), ref, f"fp8 {act}") < 1e-2
+
+
+@pytest.mark.parametrize("T", [16, 300])
+def test_fp8_graph_replay_matches_eager(T):
+    """MoEGraph (route + forward in one CUDA graph) on FP8 experts, on the
+    DECODE (T=16) and PREFILL (T=300) paths: bit-identical to eager calls."""
+    wl = G.Workload("fp8graph", T, 512, 256, 16, 4, wdtype="e4m3")
+    W = G.make_weights(wl, 0, device="cuda")
+    layer = moe.MoELayer(W["w_gate_up"], W["w_down"], wl.k, W["sw_gate_up"], W["sw_down"])
+    g = moe.MoEGraph(layer, wl.T)
+    for seed in (31, 32):
+        x, L = G.make_activations(wl, seed)
+        got = g(x.cuda(), L.cuda()).clone()
+        ref = layer(x.cuda(), L.cuda())
+        torch.cuda.synchronize()
+        assert torch.equal(got, ref)

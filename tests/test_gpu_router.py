@@ -73,3 +73,23 @@ def test_router_feeds_the_layer():
     from parity import ExpertView, assert_bf16_close
     ref = O.moe_forward(x.float().numpy(), ridx, rw, ExpertView(W["w_gate_up"]), ExpertView(W["w_down"]))
     assert_bf16_close(out.float().cpu().numpy(), ref, "router+forward")
+
+
+def test_router_in_a_cuda_graph():
+    """moe_router captured in a CUDA graph replays to the eager result."""
+    T, H, E, k = 512, 1024, 64, 4
+    wl = G.Workload("routergraph", T, H, 128, E, k)
+    w_r = G.make_router_weights(wl, 2, device="cuda")
+    x_static = torch.zeros((T, H), dtype=torch.bfloat16, device="cuda")
+    moe.router(x_static, w_r, k)  # eager warm-up (one-time set-up outside the capture)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        idx_g, w_g = moe.router(x_static, w_r, k)
+    for seed in (5, 6):
+        x, _ = G.make_activations(wl, seed)
+        x_static.copy_(x.cuda())
+        g.replay()
+        idx_e, w_e = moe.router(x.cuda(), w_r, k)
+        torch.cuda.synchronize()
+        assert torch.equal(idx_g, idx_e) and torch.equal(w_g, w_e)
