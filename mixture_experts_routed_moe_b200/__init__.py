@@ -101,6 +101,24 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
+_FLOAT8 = getattr(torch, "float8_e4m3fn", None)
+
+
+def _need(t, name, dtypes, ndim):
+    """The library reads raw device pointers: check what it cannot (type,
+    rank, contiguity, device) before handing one over."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor, got {type(t).__name__}")
+    if t.dtype not in dtypes:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected {' or '.join(str(d) for d in dtypes)}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name}: {t.dim()}-D, expected {ndim}-D")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be on a CUDA device")
+
+
 def _stream(stream=None):
     s = torch.cuda.current_stream() if stream is None else stream
     return ctypes.c_void_p(s.cuda_stream)
@@ -137,9 +155,27 @@ def route(logits: torch.Tensor, k: int, topk_idx: torch.Tensor | None = None, to
         topk_idx = torch.empty((T, k), dtype=torch.int32, device=logits.device)
     if topk_w is None:
         topk_w = torch.empty((T, k), dtype=torch.float32, device=logits.device)
-    assert logits.dtype == torch.float32 and logits.is_contiguous()
+    _need(logits, "logits", (torch.float32,), 2)
+    _need(topk_idx, "topk_idx", (torch.int32,), 2)
+    _need(topk_w, "topk_w", (torch.float32,), 2)
     _check(lib().moe_route(_ptr(logits), T, E, k, _ptr(topk_idx), _ptr(topk_w), _stream(stream)), "moe_route")
     return topk_idx, topk_w
+
+
+def _check_forward_args(x, topk_idx, topk_w, w_gate_up, w_down, sw_gate_up, sw_down, out):
+    _need(x, "x", (torch.bfloat16,), 2)
+    _need(topk_idx, "topk_idx", (torch.int32,), 2)
+    _need(topk_w, "topk_w", (torch.float32,), 2)
+    wtypes = (torch.bfloat16,) + ((_FLOAT8,) if _FLOAT8 is not None else ())
+    _need(w_gate_up, "w_gate_up", wtypes, 3)
+    _need(w_down, "w_down", (w_gate_up.dtype,), 3)
+    for name, t in (("sw_gate_up", sw_gate_up), ("sw_down", sw_down)):
+        if t is not None:
+            _need(t, name, (torch.uint8,), 3)
+    if out is not None:
+        _need(out, "out", (torch.bfloat16,), 2)
+    if topk_idx.shape != topk_w.shape or topk_idx.shape[0] != x.shape[0]:
+        raise ValueError(f"routing shapes {tuple(topk_idx.shape)}, {tuple(topk_w.shape)} do not match x {tuple(x.shape)}")
 
 
 def forward(x, topk_idx, topk_w, w_gate_up, w_down, sw_gate_up=None, sw_down=None, out=None, workspace=None,
@@ -148,6 +184,9 @@ def forward(x, topk_idx, topk_w, w_gate_up, w_down, sw_gate_up=None, sw_down=Non
     w_gate_up [E,2I,H], w_down [E,H,I] (bf16, or float8_e4m3fn with uint8 UE8M0
     block scales) -> bf16 out [T,H]; act is the gate activation ("silu" for
     SwiGLU, "gelu" for GeGLU, "relu" for ReGLU). Returns (out, workspace)."""
+    _check_forward_args(x, topk_idx, topk_w, w_gate_up, w_down, sw_gate_up, sw_down, out)
+    if workspace is not None:
+        _need(workspace, "workspace", (torch.uint8,), 1)
     T, H = x.shape
     k = topk_idx.shape[1]
     E, twoI, _ = w_gate_up.shape
@@ -176,6 +215,7 @@ def forward_noalloc(x, topk_idx, topk_w, w_gate_up, w_down, sw_gate_up=None, sw_
     array instead of a caller workspace, for callers that cannot allocate device
     memory (only ``out`` is allocated here when not given). Calls share the
     array, so calls whose GPU work overlaps must be ordered by the caller."""
+    _check_forward_args(x, topk_idx, topk_w, w_gate_up, w_down, sw_gate_up, sw_down, out)
     T, H = x.shape
     k = topk_idx.shape[1]
     E, twoI, _ = w_gate_up.shape
@@ -199,6 +239,8 @@ def router(x: torch.Tensor, w_router: torch.Tensor, k: int, logits: bool = False
     top-k routing on them, in one kernel. x bf16 [T,H], w_router bf16 [E,H].
     Returns (topk_idx int32 [T,k], topk_w fp32 [T,k]) and, with logits=True,
     the fp32 logits [T,E] as a third element."""
+    _need(x, "x", (torch.bfloat16,), 2)
+    _need(w_router, "w_router", (torch.bfloat16,), 2)
     T, H = x.shape
     E = w_router.shape[0]
     idx = torch.empty((T, k), dtype=torch.int32, device=x.device)

@@ -168,3 +168,30 @@ def test_product_code_never_touches_the_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".h")):
                 src = open(os.path.join(dirpath, f)).read()
                 assert not re.search(r"^\s*(from|import)\s+oracle|moe_oracle|oracle/", src, flags=re.M), f
+
+
+def test_binding_checks_tensor_arguments():
+    """The binding refuses what the C ABI cannot see: wrong dtype, rank,
+    layout or device (checked before anything reaches the library)."""
+    import torch
+
+    T, H, I, E, k = 4, 128, 128, 4, 2
+    x = torch.zeros((T, H), dtype=torch.bfloat16)
+    idx = torch.zeros((T, k), dtype=torch.int32)
+    w = torch.zeros((T, k), dtype=torch.float32)
+    wgu = torch.zeros((E, 2 * I, H), dtype=torch.bfloat16)
+    wd = torch.zeros((E, H, I), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="x must be on a CUDA device"):
+        moe.forward(x, idx, w, wgu, wd)
+    with pytest.raises(ValueError, match="topk_idx: dtype"):
+        moe._need(idx.long(), "topk_idx", (torch.int32,), 2)
+    with pytest.raises(ValueError, match="x: 1-D"):
+        moe._need(x[0], "x", (torch.bfloat16,), 2)
+    with pytest.raises(ValueError, match="contiguous"):
+        moe._need(wgu.transpose(1, 2), "w_gate_up", (torch.bfloat16,), 3)
+    with pytest.raises(TypeError):
+        moe._need(None, "x", (torch.bfloat16,), 2)
+    with pytest.raises(ValueError, match="logits: dtype"):
+        moe.route(torch.zeros((T, E), dtype=torch.float64), k)
+    with pytest.raises(ValueError, match="x must be on a CUDA device"):
+        moe.router(x, torch.zeros((E, H), dtype=torch.bfloat16), k)
