@@ -29,7 +29,7 @@ ACT = {"silu": 0, "gelu": 1, "relu": 2}
 PATH_NAMES = {v: k for k, v in PATH.items()}
 EXPORTS = ["moe_route", "moe_workspace_size", "moe_forward", "moe_forward_timed", "moe_workspace_query",
            "moe_read_device_status", "moe_status_string", "moe_version", "moe_forward_noalloc",
-           "moe_set_test_hooks", "moe_router"]
+           "moe_set_test_hooks", "moe_router", "moe_forward_noalloc_status"]
 
 
 class MoeError(RuntimeError):
@@ -78,6 +78,8 @@ def lib() -> ctypes.CDLL:
         L.moe_status_string.restype = ctypes.c_char_p
         L.moe_forward_noalloc.argtypes = [ctypes.POINTER(MoeShape), vp, vp, vp, vp, vp, vp, vp, vp, vp]
         L.moe_forward_noalloc.restype = i32
+        L.moe_forward_noalloc_status.argtypes = [vp]
+        L.moe_forward_noalloc_status.restype = i32
         L.moe_router.argtypes = [vp, vp, i32, i32, i32, i32, vp, vp, vp, vp]
         L.moe_router.restype = i32
         L.moe_set_test_hooks.argtypes = [i32, ctypes.c_uint64]
@@ -104,23 +106,37 @@ def _ptr(t):
 _FLOAT8 = getattr(torch, "float8_e4m3fn", None)
 
 
-def _need(t, name, dtypes, ndim):
+def _need(t, name, dtypes, ndim, shape=None, cuda=True):
     """The library reads raw device pointers: check what it cannot (type,
-    rank, contiguity, device) before handing one over."""
+    rank, sizes, contiguity, device) before handing one over. ``shape`` lists
+    the expected sizes; ``cuda`` False leaves the device to a later check."""
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor, got {type(t).__name__}")
     if t.dtype not in dtypes:
         raise ValueError(f"{name}: dtype {t.dtype}, expected {' or '.join(str(d) for d in dtypes)}")
     if t.dim() != ndim:
         raise ValueError(f"{name}: {t.dim()}-D, expected {ndim}-D")
+    if shape is not None and tuple(t.shape) != tuple(int(v) for v in shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(int(v) for v in shape)}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
-    if not t.is_cuda:
+    if cuda and not t.is_cuda:
         raise ValueError(f"{name} must be on a CUDA device")
 
 
-def _stream(stream=None):
-    s = torch.cuda.current_stream() if stream is None else stream
+def _same_device(device, **tensors):
+    """Every tensor on ``device`` (a CUDA device): the library launches on the
+    current device and stream, so one tensor elsewhere would be read from the
+    wrong GPU."""
+    if device.type != "cuda":
+        raise ValueError(f"x must be on a CUDA device, not {device}")
+    for name, t in tensors.items():
+        if t is not None and t.device != device:
+            raise ValueError(f"{name} is on {t.device}, x on {device}: all tensors must share one CUDA device")
+
+
+def _stream(stream=None, device=None):
+    s = torch.cuda.current_stream(device) if stream is None else stream
     return ctypes.c_void_p(s.cuda_stream)
 
 
@@ -150,32 +166,57 @@ def alloc_workspace(shape: MoeShape, device=None) -> torch.Tensor:
 def route(logits: torch.Tensor, k: int, topk_idx: torch.Tensor | None = None, topk_w: torch.Tensor | None = None,
           stream=None):
     """moe_route: fp32 logits [T,E] -> (int32 [T,k], fp32 [T,k])."""
+    _need(logits, "logits", (torch.float32,), 2, cuda=False)
     T, E = logits.shape
     if topk_idx is None:
         topk_idx = torch.empty((T, k), dtype=torch.int32, device=logits.device)
     if topk_w is None:
         topk_w = torch.empty((T, k), dtype=torch.float32, device=logits.device)
-    _need(logits, "logits", (torch.float32,), 2)
-    _need(topk_idx, "topk_idx", (torch.int32,), 2)
-    _need(topk_w, "topk_w", (torch.float32,), 2)
-    _check(lib().moe_route(_ptr(logits), T, E, k, _ptr(topk_idx), _ptr(topk_w), _stream(stream)), "moe_route")
+    _need(topk_idx, "topk_idx", (torch.int32,), 2, (T, k), cuda=False)
+    _need(topk_w, "topk_w", (torch.float32,), 2, (T, k), cuda=False)
+    _same_device(logits.device, topk_idx=topk_idx, topk_w=topk_w)
+    with torch.cuda.device(logits.device):
+        _check(lib().moe_route(_ptr(logits), T, E, k, _ptr(topk_idx), _ptr(topk_w), _stream(stream, logits.device)),
+               "moe_route")
     return topk_idx, topk_w
 
 
-def _check_forward_args(x, topk_idx, topk_w, w_gate_up, w_down, sw_gate_up, sw_down, out):
-    _need(x, "x", (torch.bfloat16,), 2)
-    _need(topk_idx, "topk_idx", (torch.int32,), 2)
-    _need(topk_w, "topk_w", (torch.float32,), 2)
+def _check_forward_args(x, topk_idx, topk_w, w_gate_up, w_down, sw_gate_up, sw_down, out, workspace=None):
+    """Checks every tensor of a forward call against the layer the weights
+    define (E experts, [gate; up] rows 2I, hidden H, top-k from topk_idx) and
+    returns (T, H, I, E, k, wdtype). Sizes first, then that all share x's CUDA
+    device: nothing reaches the library unless every pointer covers the
+    extent the kernels will read or write."""
+    _need(x, "x", (torch.bfloat16,), 2, cuda=False)
+    T, H = x.shape
+    _need(topk_idx, "topk_idx", (torch.int32,), 2, cuda=False)
+    k = topk_idx.shape[1]
+    _need(topk_idx, "topk_idx", (torch.int32,), 2, (T, k), cuda=False)
+    _need(topk_w, "topk_w", (torch.float32,), 2, (T, k), cuda=False)
     wtypes = (torch.bfloat16,) + ((_FLOAT8,) if _FLOAT8 is not None else ())
-    _need(w_gate_up, "w_gate_up", wtypes, 3)
-    _need(w_down, "w_down", (w_gate_up.dtype,), 3)
-    for name, t in (("sw_gate_up", sw_gate_up), ("sw_down", sw_down)):
-        if t is not None:
-            _need(t, name, (torch.uint8,), 3)
+    _need(w_gate_up, "w_gate_up", wtypes, 3, cuda=False)
+    E, twoI = w_gate_up.shape[0], w_gate_up.shape[1]
+    if twoI % 2 != 0:
+        raise ValueError(f"w_gate_up: {twoI} rows per expert, expected 2*I (gate rows, then up rows)")
+    I = twoI // 2
+    _need(w_gate_up, "w_gate_up", wtypes, 3, (E, 2 * I, H), cuda=False)
+    _need(w_down, "w_down", (w_gate_up.dtype,), 3, (E, H, I), cuda=False)
+    fp8 = _FLOAT8 is not None and w_gate_up.dtype == _FLOAT8
+    if fp8:
+        # UE8M0 bytes, one per 128x128 weight block (None: the library refuses with MOE_ERR_SCALE_FORMAT)
+        if sw_gate_up is not None:
+            _need(sw_gate_up, "sw_gate_up", (torch.uint8,), 3, (E, 2 * I // 128, H // 128), cuda=False)
+        if sw_down is not None:
+            _need(sw_down, "sw_down", (torch.uint8,), 3, (E, H // 128, I // 128), cuda=False)
+    elif sw_gate_up is not None or sw_down is not None:
+        raise ValueError("block scales were given for bf16 experts")
     if out is not None:
-        _need(out, "out", (torch.bfloat16,), 2)
-    if topk_idx.shape != topk_w.shape or topk_idx.shape[0] != x.shape[0]:
-        raise ValueError(f"routing shapes {tuple(topk_idx.shape)}, {tuple(topk_w.shape)} do not match x {tuple(x.shape)}")
+        _need(out, "out", (torch.bfloat16,), 2, (T, H), cuda=False)
+    if workspace is not None:
+        _need(workspace, "workspace", (torch.uint8,), 1, cuda=False)
+    _same_device(x.device, topk_idx=topk_idx, topk_w=topk_w, w_gate_up=w_gate_up, w_down=w_down,
+                 sw_gate_up=sw_gate_up, sw_down=sw_down, out=out, workspace=workspace)
+    return T, H, I, E, k, ("e4m3" if fp8 else "bf16")
 
 
 def forward(x, topk_idx, topk_w, w_gate_up, w_down, sw_gate_up=None, sw_down=None, out=None, workspace=None,
@@ -184,28 +225,25 @@ def forward(x, topk_idx, topk_w, w_gate_up, w_down, sw_gate_up=None, sw_down=Non
     w_gate_up [E,2I,H], w_down [E,H,I] (bf16, or float8_e4m3fn with uint8 UE8M0
     block scales) -> bf16 out [T,H]; act is the gate activation ("silu" for
     SwiGLU, "gelu" for GeGLU, "relu" for ReGLU). Returns (out, workspace)."""
-    _check_forward_args(x, topk_idx, topk_w, w_gate_up, w_down, sw_gate_up, sw_down, out)
-    if workspace is not None:
-        _need(workspace, "workspace", (torch.uint8,), 1)
-    T, H = x.shape
-    k = topk_idx.shape[1]
-    E, twoI, _ = w_gate_up.shape
-    wdtype = "e4m3" if w_gate_up.dtype == torch.float8_e4m3fn else "bf16"
-    shape = make_shape(T, H, twoI // 2, E, k, wdtype, path, act)
-    if out is None:
-        out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device)
-    if workspace is None:
-        workspace = alloc_workspace(shape, x.device)
-    args = [ctypes.byref(shape), _ptr(x), _ptr(topk_idx), _ptr(topk_w), _ptr(w_gate_up), _ptr(w_down),
-            _ptr(sw_gate_up), _ptr(sw_down), _ptr(out), _ptr(workspace), workspace.numel(), _stream(stream)]
-    if events is None:
-        _check(lib().moe_forward(*args), "moe_forward")
-    else:
-        for e in events:  # torch creates the CUDA event lazily, on its first record
-            if not e.cuda_event:
-                e.record(stream or torch.cuda.current_stream())
-        ev = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
-        _check(lib().moe_forward_timed(*args, ev, len(events)), "moe_forward_timed")
+    T, H, I, E, k, wdtype = _check_forward_args(x, topk_idx, topk_w, w_gate_up, w_down, sw_gate_up, sw_down, out,
+                                                workspace)
+    shape = make_shape(T, H, I, E, k, wdtype, path, act)
+    with torch.cuda.device(x.device):
+        if out is None:
+            out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device)
+        if workspace is None:
+            workspace = alloc_workspace(shape, x.device)
+        st = stream or torch.cuda.current_stream(x.device)
+        args = [ctypes.byref(shape), _ptr(x), _ptr(topk_idx), _ptr(topk_w), _ptr(w_gate_up), _ptr(w_down),
+                _ptr(sw_gate_up), _ptr(sw_down), _ptr(out), _ptr(workspace), workspace.numel(), _stream(st)]
+        if events is None:
+            _check(lib().moe_forward(*args), "moe_forward")
+        else:
+            for e in events:  # torch creates the CUDA event lazily, on its first record
+                if not e.cuda_event:
+                    e.record(st)
+            ev = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+            _check(lib().moe_forward_timed(*args, ev, len(events)), "moe_forward_timed")
     return out, workspace
 
 
@@ -215,23 +253,30 @@ def forward_noalloc(x, topk_idx, topk_w, w_gate_up, w_down, sw_gate_up=None, sw_
     array instead of a caller workspace, for callers that cannot allocate device
     memory (only ``out`` is allocated here when not given). Calls share the
     array, so calls whose GPU work overlaps must be ordered by the caller."""
-    _check_forward_args(x, topk_idx, topk_w, w_gate_up, w_down, sw_gate_up, sw_down, out)
-    T, H = x.shape
-    k = topk_idx.shape[1]
-    E, twoI, _ = w_gate_up.shape
-    wdtype = "e4m3" if w_gate_up.dtype == torch.float8_e4m3fn else "bf16"
-    shape = make_shape(T, H, twoI // 2, E, k, wdtype, path, act)
-    if out is None:
-        out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device)
-    _check(lib().moe_forward_noalloc(ctypes.byref(shape), _ptr(x), _ptr(topk_idx), _ptr(topk_w), _ptr(w_gate_up),
-                                     _ptr(w_down), _ptr(sw_gate_up), _ptr(sw_down), _ptr(out), _stream(stream)),
-           "moe_forward_noalloc")
+    T, H, I, E, k, wdtype = _check_forward_args(x, topk_idx, topk_w, w_gate_up, w_down, sw_gate_up, sw_down, out)
+    shape = make_shape(T, H, I, E, k, wdtype, path, act)
+    with torch.cuda.device(x.device):
+        if out is None:
+            out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device)
+        _check(lib().moe_forward_noalloc(ctypes.byref(shape), _ptr(x), _ptr(topk_idx), _ptr(topk_w),
+                                         _ptr(w_gate_up), _ptr(w_down), _ptr(sw_gate_up), _ptr(sw_down), _ptr(out),
+                                         _stream(stream, x.device)),
+               "moe_forward_noalloc")
     return out
+
+
+def noalloc_device_status(device=None, stream=None) -> int:
+    """Synchronises the stream and returns the device status of the last
+    forward_noalloc on `device` (read from the library's own scratch)."""
+    device = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    with torch.cuda.device(device):
+        return int(lib().moe_forward_noalloc_status(_stream(stream, device)))
 
 
 def read_device_status(workspace: torch.Tensor, stream=None) -> int:
     """Synchronises the stream and returns the device status of the last forward on `workspace`."""
-    return int(lib().moe_read_device_status(_ptr(workspace), _stream(stream)))
+    with torch.cuda.device(workspace.device):
+        return int(lib().moe_read_device_status(_ptr(workspace), _stream(stream, workspace.device)))
 
 
 def router(x: torch.Tensor, w_router: torch.Tensor, k: int, logits: bool = False, stream=None):
@@ -239,15 +284,19 @@ def router(x: torch.Tensor, w_router: torch.Tensor, k: int, logits: bool = False
     top-k routing on them, in one kernel. x bf16 [T,H], w_router bf16 [E,H].
     Returns (topk_idx int32 [T,k], topk_w fp32 [T,k]) and, with logits=True,
     the fp32 logits [T,E] as a third element."""
-    _need(x, "x", (torch.bfloat16,), 2)
-    _need(w_router, "w_router", (torch.bfloat16,), 2)
+    _need(x, "x", (torch.bfloat16,), 2, cuda=False)
     T, H = x.shape
+    _need(w_router, "w_router", (torch.bfloat16,), 2, cuda=False)
     E = w_router.shape[0]
-    idx = torch.empty((T, k), dtype=torch.int32, device=x.device)
-    w = torch.empty((T, k), dtype=torch.float32, device=x.device)
-    lg = torch.empty((T, E), dtype=torch.float32, device=x.device) if logits else None
-    _check(lib().moe_router(_ptr(x), _ptr(w_router), T, H, E, k, _ptr(lg), _ptr(idx), _ptr(w), _stream(stream)),
-           "moe_router")
+    _need(w_router, "w_router", (torch.bfloat16,), 2, (E, H), cuda=False)
+    _same_device(x.device, w_router=w_router)
+    with torch.cuda.device(x.device):
+        idx = torch.empty((T, k), dtype=torch.int32, device=x.device)
+        w = torch.empty((T, k), dtype=torch.float32, device=x.device)
+        lg = torch.empty((T, E), dtype=torch.float32, device=x.device) if logits else None
+        _check(lib().moe_router(_ptr(x), _ptr(w_router), T, H, E, k, _ptr(lg), _ptr(idx), _ptr(w),
+                                _stream(stream, x.device)),
+               "moe_router")
     return (idx, w, lg) if logits else (idx, w)
 
 
@@ -322,6 +371,6 @@ class MoEGraph:
         return self.replay()
 
 
-__all__ = ["lib", "route", "forward", "forward_noalloc", "MoEGraph", "workspace_size", "workspace_layout", "alloc_workspace",
+__all__ = ["lib", "route", "forward", "forward_noalloc", "noalloc_device_status", "MoEGraph", "workspace_size", "workspace_layout", "alloc_workspace",
            "read_device_status", "set_test_hooks", "router", "make_shape", "MoELayer", "MoeError", "MoeShape", "EXPORTS", "STATUS",
            "status_string", "PATH", "WDTYPE", "ACT"]

@@ -48,7 +48,7 @@ def shape(**kw):
     return moe.make_shape(**d)
 
 
-@pytest.mark.parametrize("bad", [dict(H=100), dict(I=64), dict(E=0), dict(E=1025), dict(k=0), dict(k=9),
+@pytest.mark.parametrize("bad", [dict(H=100), dict(I=96), dict(E=0), dict(E=1025), dict(k=0), dict(k=9),
                                  dict(T=-1), dict(wdtype=7), dict(path=9), dict(H=0), dict(act=3)])
 def test_invalid_shapes_rejected(L, bad):
     s = shape(**bad)
@@ -56,6 +56,20 @@ def test_invalid_shapes_rejected(L, bad):
     lay = moe.MoeWorkspaceLayout()
     assert L.moe_workspace_query(ctypes.byref(s), ctypes.byref(lay)) == -1
     r = L.moe_forward(ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, FAKE, None, None, FAKE, FAKE, 1 << 40, None)
+    assert r == -1
+
+
+@pytest.mark.parametrize("H,I", [(128, 64), (192, 256), (64, 64)])
+def test_bf16_64_aligned_sizes_are_unsupported_not_invalid(L, H, I):
+    """bf16 layers with H, I multiples of 64 but not of 128 are valid requests
+    this build does not run: MOE_ERR_UNSUPPORTED, not MOE_ERR_INVALID_ARG;
+    the same sizes with e4m3 experts are invalid (FP8 needs 128-wide blocks)."""
+    s = shape(H=H, I=I)
+    r = L.moe_forward(ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, FAKE, None, None, FAKE, FAKE, 1 << 40, None)
+    assert r == -2
+    assert L.moe_workspace_size(ctypes.byref(s)) == 0
+    s = shape(H=H, I=I, wdtype="e4m3")
+    r = L.moe_forward(ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 40, None)
     assert r == -1
 
 
@@ -195,3 +209,67 @@ def test_binding_checks_tensor_arguments():
         moe.route(torch.zeros((T, E), dtype=torch.float64), k)
     with pytest.raises(ValueError, match="x must be on a CUDA device"):
         moe.router(x, torch.zeros((E, H), dtype=torch.bfloat16), k)
+
+
+def test_binding_checks_sizes_before_any_launch():
+    """Every tensor's sizes are checked against the layer that x, topk_idx and
+    w_gate_up define, so no kernel can read or write past an allocation
+    (checked on the host, before the device check and before the library)."""
+    import torch
+
+    T, H, I, E, k = 4, 128, 128, 4, 2
+    bf = torch.bfloat16
+    ok = dict(x=torch.zeros((T, H), dtype=bf), topk_idx=torch.zeros((T, k), dtype=torch.int32),
+              topk_w=torch.zeros((T, k), dtype=torch.float32), w_gate_up=torch.zeros((E, 2 * I, H), dtype=bf),
+              w_down=torch.zeros((E, H, I), dtype=bf))
+
+    def call(**bad):
+        a = dict(ok)
+        a.update(bad)
+        return moe.forward(**a)
+
+    cases = [
+        (dict(w_gate_up=torch.zeros((E, 2 * I, H + 128), dtype=bf)), "w_gate_up: shape"),
+        (dict(w_gate_up=torch.zeros((E, 2 * I + 1, H), dtype=bf)), "2\\*I"),
+        (dict(w_down=torch.zeros((E, H, 2 * I), dtype=bf)), "w_down: shape"),
+        (dict(w_down=torch.zeros((E + 1, H, I), dtype=bf)), "w_down: shape"),
+        (dict(topk_w=torch.zeros((T, k + 1), dtype=torch.float32)), "topk_w: shape"),
+        (dict(topk_idx=torch.zeros((T + 1, k), dtype=torch.int32)), "topk_idx: shape"),
+        (dict(out=torch.zeros((T, H - 8), dtype=bf)), "out: shape"),
+        (dict(sw_gate_up=torch.zeros((E, 2, 1), dtype=torch.uint8)), "bf16 experts"),
+        (dict(workspace=torch.zeros((8, 8), dtype=torch.uint8)), "workspace: 2-D"),
+    ]
+    for bad, msg in cases:
+        with pytest.raises(ValueError, match=msg):
+            call(**bad)
+    # e4m3 experts: the UE8M0 block grids must match the weights
+    f8 = torch.float8_e4m3fn
+    e4 = dict(w_gate_up=torch.zeros((E, 2 * I, H), dtype=f8), w_down=torch.zeros((E, H, I), dtype=f8))
+    with pytest.raises(ValueError, match="sw_gate_up: shape"):
+        call(**e4, sw_gate_up=torch.zeros((E, 2 * I // 128, H // 128 + 1), dtype=torch.uint8),
+             sw_down=torch.zeros((E, H // 128, I // 128), dtype=torch.uint8))
+    with pytest.raises(ValueError, match="sw_down: shape"):
+        call(**e4, sw_gate_up=torch.zeros((E, 2 * I // 128, H // 128), dtype=torch.uint8),
+             sw_down=torch.zeros((E, I // 128, H // 128 + 1), dtype=torch.uint8))
+    with pytest.raises(ValueError, match="w_down: dtype"):
+        call(w_gate_up=torch.zeros((E, 2 * I, H), dtype=f8))
+    # well-formed arguments get as far as the device check
+    with pytest.raises(ValueError, match="x must be on a CUDA device"):
+        call()
+    with pytest.raises(ValueError, match="w_router: shape"):
+        moe.router(ok["x"], torch.zeros((E, H + 64), dtype=bf), k)
+    with pytest.raises(ValueError, match="topk_w: shape"):
+        moe.route(torch.zeros((T, E), dtype=torch.float32), k, topk_w=torch.zeros((T, k + 1)))
+
+
+def test_binding_requires_one_device():
+    """A tensor on another device than x is refused (the library launches on
+    the current device only)."""
+    import torch
+
+    dev = torch.device("cuda", 0)
+    with pytest.raises(ValueError, match="w_down is on cpu"):
+        moe._same_device(dev, w_down=torch.zeros(1))
+    with pytest.raises(ValueError, match="on a CUDA device"):
+        moe._same_device(torch.device("cpu"))
+    moe._same_device(dev, out=None)  # absent tensors are fine
