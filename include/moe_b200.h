@@ -67,7 +67,11 @@ typedef enum {
 
 /* Problem shape. T tokens, hidden size H, expert intermediate size I,
  * E experts, top-k. Requirements: T >= 0; H and I positive multiples of 128;
- * 1 <= E <= 1024; 1 <= k <= E; T*k < 2^31 and every buffer below 2^31 rows. */
+ * 1 <= E <= 1024; 1 <= k <= E; T*k < 2^31 and every buffer below 2^31 rows.
+ * bf16 experts whose H and I are multiples of 64 but not both of 128 form a
+ * valid layer that this build does not run: moe_forward returns
+ * MOE_ERR_UNSUPPORTED for them (and moe_workspace_size 0); other sizes are
+ * MOE_ERR_INVALID_ARG. */
 typedef struct {
   int32_t T, H, I, E, k;
   int32_t wdtype; /* moe_wdtype */
@@ -224,12 +228,21 @@ moe_status moe_set_test_hooks(int32_t stall_gate_up_loads, uint64_t wait_limit_n
  *    that device current); make that first call before any stream capture.
  *  - All calls share the one array and leave their intermediates in it. Calls
  *    whose GPU work overlaps in time race on it: order them, for example by
- *    issuing them on one stream. moe_read_device_status does not apply here.
+ *    issuing them on one stream. Device-side errors are read with
+ *    moe_forward_noalloc_status (moe_read_device_status takes a workspace).
  */
 #define MOE_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20) /* 8 MiB */
 moe_status moe_forward_noalloc(const moe_shape* shape, const void* x, const int32_t* topk_idx,
                                const float* topk_w, const void* w_gate_up, const void* w_down,
                                const uint8_t* sw_gate_up, const uint8_t* sw_down, void* out, void* stream);
+
+/* The device status of the last moe_forward_noalloc on the current device
+ * (the counterpart of moe_read_device_status for the library's own scratch):
+ * synchronises `stream`, then returns MOE_OK, MOE_ERR_DEVICE_INDEX or
+ * MOE_ERR_DEVICE_TIMEOUT (MOE_ERR_CUDA if the read fails). Allocates nothing.
+ * Like the forward's scratch, the word is shared by every call on the device:
+ * read it after the call it should describe and before the next one. */
+moe_status moe_forward_noalloc_status(void* stream);
 
 /* Static description of a status code (never NULL). */
 const char* moe_status_string(moe_status status);

@@ -201,10 +201,19 @@ using namespace moe;
 
 namespace {
 
+// bf16 experts whose H and I are multiples of 64 but not both of 128: a valid
+// layer (the boundary accepts 64-aligned bf16 sizes) that this build's
+// 128-wide tiles do not cover.
+bool bf16_64_not_128(const moe_shape* s) {
+  if (s == nullptr || s->wdtype != MOE_DT_BF16 || s->H < 64 || s->I < 64) return false;
+  return s->H % 64 == 0 && s->I % 64 == 0 && (s->H % 128 != 0 || s->I % 128 != 0);
+}
+
 moe_status forward_impl(const moe_shape* shape, const void* x, const int32_t* topk_idx, const float* topk_w,
                         const void* w_gate_up, const void* w_down, const uint8_t* sw_gate_up,
                         const uint8_t* sw_down, void* out, void* workspace, size_t workspace_bytes, void* stream,
                         void* const* events, int32_t n_events) {
+  if (bf16_64_not_128(shape)) return MOE_ERR_UNSUPPORTED;
   if (!validate_shape(shape)) return MOE_ERR_INVALID_ARG;
   if (!(n_events == 0 || (n_events == 5 && events != nullptr))) return MOE_ERR_INVALID_ARG;
   const bool fp8 = shape->wdtype == MOE_DT_E4M3;
