@@ -112,15 +112,27 @@ def e4m3_encode(v) -> np.ndarray:
     return (code.astype(np.uint8) | sign).astype(np.uint8)
 
 
-def e4m3_decode(codes) -> np.ndarray:
-    """Float64 values of e4m3 byte codes (0x7F/0xFF are NaN)."""
-    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+def _e4m3_value(c) -> np.ndarray:
+    """Float64 value of each e4m3 byte code: sign bit 7, exponent field e (bits
+    6..3, bias 7), mantissa m (bits 2..0); e = 0 is subnormal m * 2^-9,
+    otherwise (1 + m/8) * 2^(e-7); 0x7F and 0xFF are NaN."""
+    c = np.asarray(c, dtype=np.uint8).astype(np.int64)
     s = np.where(c & 0x80, -1.0, 1.0)
     e = (c >> 3) & 0xF
     m = c & 0x7
     val = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * np.ldexp(1.0, e - 7))
     val = np.where((c & 0x7F) == 0x7F, np.nan, val)
     return s * val
+
+
+# the 256 values, one per code, so that decoding a large matrix is one lookup
+_E4M3_VALUES = _e4m3_value(np.arange(256, dtype=np.uint8))
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    """Float64 values of e4m3 byte codes (0x7F/0xFF are NaN): the value of
+    each code, looked up in the table of all 256."""
+    return _E4M3_VALUES[np.asarray(codes, dtype=np.uint8)]
 
 
 def ue8m0_scale(b) -> np.ndarray:
@@ -279,6 +291,42 @@ def combine(Y, topk_w, intermediate: str = "bf16"):
     return bf16_round(out) if intermediate in ("bf16", "exact") else out
 
 
+def fma_f32(a, b, c) -> np.ndarray:
+    """Single-precision fused multiply-add, round(a*b + c) to the nearest
+    float32 (ties to even), for float32-valued inputs; returns float64.
+
+    The product of two float32 values has at most 48 significant bits, so a*b
+    is exact in float64. The sum is split exactly into s + err (Knuth's
+    TwoSum); s is then moved to its odd neighbour when err is nonzero and s is
+    even (rounding to odd), after which one rounding to float32 is the correct
+    one: float64 carries more than 24 + 1 extra bits, so no double rounding."""
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    c = np.asarray(c, dtype=np.float64)
+    p = a * b
+    s = p + c
+    bv = s - p
+    err = (p - (s - bv)) + (c - bv)
+    even = (s.view(np.int64) & 1) == 0
+    toward = np.where(err > 0, np.inf, -np.inf)
+    s = np.where((err != 0) & even, np.nextafter(s, toward), s)
+    return s.astype(np.float32).astype(np.float64)
+
+
+def combine_fp32_fma(Y, topk_w):
+    """The aggregation of reading R5 in the precision the boundary states:
+    acc = 0 in float32, then acc = fma(w[t,j], Y[t,j], acc) for j = 0..k-1 in
+    ascending order, and the output rounded to bf16 once at the end
+    (introduction: the routing-weighted sum of the experts' results). With the
+    same Y this fixes every bit of the output."""
+    w = np.asarray(topk_w, dtype=np.float32).astype(np.float64)
+    Y = np.asarray(Y, dtype=np.float64)
+    acc = np.zeros((Y.shape[0], Y.shape[2]), dtype=np.float64)
+    for j in range(Y.shape[1]):
+        acc = fma_f32(w[:, j:j + 1], Y[:, j], acc)
+    return bf16_round(acc)
+
+
 def moe_forward(x, topk_idx, topk_w, w_gate_up, w_down, intermediate: str = "bf16",
                 tokens=None, act: str = "silu"):
     """Routed MoE forward for bf16 experts.
@@ -315,7 +363,10 @@ def dequantize_blocks(codes, scale_bytes):
     scales on Blackwell)."""
     q = e4m3_decode(codes)
     s = ue8m0_scale(scale_bytes)
-    return q * np.repeat(np.repeat(s, QBLOCK, axis=0), QBLOCK, axis=1)
+    R, C = q.shape
+    # element (r, c) takes the scale of block (r // 128, c // 128)
+    q4 = q.reshape(R // QBLOCK, QBLOCK, C // QBLOCK, QBLOCK)
+    return (q4 * s[:, None, :, None]).reshape(R, C)
 
 
 def quantize_1x128(a):

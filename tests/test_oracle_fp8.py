@@ -97,3 +97,34 @@ def test_fp8_forward_without_activation_quant_equals_dequantised_bf16_forward():
                           W["sw_down"].numpy(), quantize_acts=True)
     rel_q = np.linalg.norm(c - b) / np.linalg.norm(b)
     assert 1e-2 < rel_q < 2 * 2.0 ** -4
+
+
+def test_fp8_h_quantised_from_fp32_hand_worked(golden):
+    """h is quantised 1x128 from its fp32 value (reading R7), not from a bf16
+    copy: a hand-worked ReLU case where h = 1.064453125 rounds to e4m3 1.125,
+    while its bf16 value 1.0625 is an exact e4m3 midpoint that rounds to 1.0."""
+    c = golden("rounding_points.json")["fp8_h_from_fp32"]
+    H, I = c["H"], c["I"]
+    x = np.zeros((1, H))
+    for col, v in c["x_nonzero"]:
+        x[0, col] = v
+    wgu = np.zeros((2 * I, H), dtype=np.uint8)
+    for r, col, code in c["w_gate_up_codes"]:
+        wgu[r, col] = code
+    wd = np.zeros((H, I), dtype=np.uint8)
+    for r, col, code in c["w_down_codes"]:
+        wd[r, col] = code
+    sgu = np.full((2 * I // 128, H // 128), c["scale_byte"], dtype=np.uint8)
+    sd = np.full((H // 128, I // 128), c["scale_byte"], dtype=np.uint8)
+    y = O.expert_mlp_fp8(x, wgu, sgu, wd, sd, act=c["act"])
+    want = np.zeros((1, H))
+    for col, v in c["y_nonzero"]:
+        want[0, col] = v
+    assert np.array_equal(y, want)
+    assert y[0, 0] != c["y0_if_h_quantised_from_bf16"]
+    # the h codes the hand derivation names, from the activation quantiser itself
+    h = np.zeros((1, I), dtype=np.float32)
+    h[0, 0], h[0, 1] = 448.0, 1.064453125
+    codes, scales, _ = O.quantize_1x128(h)
+    assert scales[0, 0] == 1.0
+    assert [(int(i), int(codes[0, i])) for i in np.nonzero(codes[0])[0]] == [tuple(v) for v in c["h_codes_nonzero"]]

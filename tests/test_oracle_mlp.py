@@ -157,3 +157,26 @@ def test_gated_activation_forward_matches_batched(act):
             h = f(torch.from_numpy(wgu[e, :I]) @ xt) * (torch.from_numpy(wgu[e, I:]) @ xt)
             ref[t] += float(w[t, j]) * (torch.from_numpy(wd[e]) @ h).numpy()
     np.testing.assert_allclose(out, ref, rtol=1e-11, atol=1e-12)
+
+
+def test_bf16_rounding_points_hand_worked(golden):
+    """h is rounded to bf16 before the down projection and y is rounded to
+    bf16 (reading R4): a hand-worked ReLU case whose exact values sit so that
+    dropping either rounding, or moving it, changes y."""
+    c = golden("rounding_points.json")["bf16_intermediates"]
+    x = np.array(c["x"], dtype=np.float64)
+    wgu = np.array(c["w_gate_up"], dtype=np.float64)
+    wd = np.array(c["w_down"], dtype=np.float64)
+    h, y = O.expert_mlp(x, wgu, wd, "bf16", act=c["act"])
+    assert np.array_equal(h, np.array(c["h"]))
+    assert np.array_equal(y, np.array(c["y"]))
+    # the case separates the readings: each wrong rounding point gives another y
+    assert not np.array_equal(np.array(c["y"]), np.array(c["y_if_h_not_rounded"]))
+    assert not np.array_equal(np.array(c["y"]), np.array(c["y_if_y_not_rounded"]))
+    # "exact" mode (no intermediate rounding) lands on neither rounded value
+    _, y_exact = O.expert_mlp(x, wgu, wd, "exact", act=c["act"])
+    assert y_exact[0, 0] != c["y"][0][0]
+    # through the whole layer (E=1, k=1, w=1): the output is bf16(y) = y
+    out = O.moe_forward(x, np.zeros((1, 1), np.int32), np.ones((1, 1), np.float32), wgu[None], wd[None],
+                        act=c["act"])
+    assert np.array_equal(out, np.array(c["y"]))
