@@ -43,19 +43,27 @@ def assert_fp8_close(got, ref, what=""):
 
 class ExpertView:
     """Per-expert host copies of device expert weights, made on first use, so
-    the oracle can index w[e] without copying experts nobody selected."""
+    the oracle can index w[e] without copying experts nobody selected. With
+    cache=False each access copies again and nothing is kept (the full-size
+    layers' weights would not fit in host memory twice over)."""
 
-    def __init__(self, t: torch.Tensor, as_codes: bool = False):
+    def __init__(self, t: torch.Tensor, as_codes: bool = False, cache: bool = True):
         self.t = t
         self.shape = tuple(t.shape)
         self.as_codes = as_codes
+        self.cache = cache
         self._cache = {}
+
+    def _copy(self, e):
+        v = self.t[e].cpu()
+        return v.view(torch.uint8).numpy() if self.as_codes else v.float().numpy()
 
     def __getitem__(self, e):
         e = int(e)
+        if not self.cache:
+            return self._copy(e)
         if e not in self._cache:
-            v = self.t[e].cpu()
-            self._cache[e] = v.view(torch.uint8).numpy() if self.as_codes else v.float().numpy()
+            self._cache[e] = self._copy(e)
         return self._cache[e]
 
 
@@ -88,12 +96,42 @@ def device_inputs(wl: G.Workload, seed: int, weights_device="cuda"):
     return x, logits, W
 
 
-def oracle_forward_bf16(x_cpu, idx, w, W, tokens=None, intermediate="bf16"):
-    return O.moe_forward(x_cpu.float().numpy(), idx, w, ExpertView(W["w_gate_up"]), ExpertView(W["w_down"]),
-                         intermediate=intermediate, tokens=tokens)
+def oracle_forward_bf16(x_cpu, idx, w, W, tokens=None, intermediate="bf16", cache=True):
+    return O.moe_forward(x_cpu.float().numpy(), idx, w, ExpertView(W["w_gate_up"], cache=cache),
+                         ExpertView(W["w_down"], cache=cache), intermediate=intermediate, tokens=tokens)
 
 
-def oracle_forward_fp8(x_cpu, idx, w, W, tokens=None):
-    return O.moe_forward_fp8(x_cpu.float().numpy(), idx, w, ExpertView(W["w_gate_up"], True),
-                             ExpertView(W["sw_gate_up"], True), ExpertView(W["w_down"], True),
-                             ExpertView(W["sw_down"], True), tokens=tokens)
+def oracle_forward_fp8(x_cpu, idx, w, W, tokens=None, cache=True):
+    return O.moe_forward_fp8(x_cpu.float().numpy(), idx, w, ExpertView(W["w_gate_up"], True, cache),
+                             ExpertView(W["sw_gate_up"], True, cache), ExpertView(W["w_down"], True, cache),
+                             ExpertView(W["sw_down"], True, cache), tokens=tokens)
+
+
+def check_combine_bit_exact(ws, shape, topk_w_np, out, chunk=1024):
+    """The device combine against the oracle's fixed-order fp32 combine on the
+    expert outputs y the device itself produced (read from the workspace):
+    every output bit must agree."""
+    lay = moe.workspace_layout(shape)
+    T, k, H = shape.T, shape.k, shape.H
+    slot = ws_i32(ws, lay.slot_row, T * k).reshape(T, k)
+    y_all = ws[lay.y:lay.y + 2 * lay.m_rows * H].view(torch.bfloat16).reshape(lay.m_rows, H)
+    got = out.float().cpu().numpy()
+    for t0 in range(0, T, chunk):
+        t1 = min(T, t0 + chunk)
+        rows = torch.from_numpy(slot[t0:t1].reshape(-1).astype(np.int64)).to(y_all.device)
+        Y = y_all.index_select(0, rows).float().cpu().numpy().reshape(t1 - t0, k, H)
+        ref = O.combine_fp32_fma(Y, topk_w_np[t0:t1])
+        bad = np.nonzero(got[t0:t1] != ref)
+        assert bad[0].size == 0, f"combine differs at {bad[0].size} elements, first token {t0 + bad[0][0]}"
+
+
+def assert_tokens_close(got, ref, bound, what=""):
+    """Per-token relative error (Frobenius over the token's H outputs) at most
+    `bound`: a check that no single token is wrong, which the whole-layer norm
+    could hide among thousands of good ones."""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    num = np.linalg.norm(got - ref, axis=1)
+    den = np.maximum(np.linalg.norm(ref, axis=1), 1e-300)
+    worst = int(np.argmax(num / den))
+    assert (num / den).max() <= bound, f"{what}: token {worst} rel_fro={num[worst] / den[worst]:.3e}"

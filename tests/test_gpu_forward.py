@@ -10,8 +10,8 @@ import mixture_experts_routed_moe_b200 as moe
 from mixture_experts_routed_moe_b200 import inputs as G
 from oracle import moe_oracle as O
 
-from parity import (ExpertView, assert_bf16_close, check_permutation, device_inputs, oracle_forward_bf16,
-                    ws_bf16)
+from parity import (ExpertView, assert_bf16_close, assert_tokens_close, check_combine_bit_exact,
+                    check_permutation, device_inputs, oracle_forward_bf16, ws_bf16)
 
 pytestmark = pytest.mark.gpu
 
@@ -86,7 +86,9 @@ def test_edge_counts(T, H, I, E, k, counts, path):
     wl = G.Workload("edge", T, H, I, E, k)
     idx, w = G.routed_inputs_with_counts(wl, counts, seed=T)
     x, idx_np, w_np, W, out, ws = _forward(wl, 3, path, idx=idx, w=w)
-    check_permutation(ws, moe.make_shape(T, H, I, E, k, "bf16", path), idx_np)
+    shape = moe.make_shape(T, H, I, E, k, "bf16", path)
+    check_permutation(ws, shape, idx_np)
+    check_combine_bit_exact(ws, shape, w_np, out)
     ref = oracle_forward_bf16(x, idx_np, w_np, W)
     assert_bf16_close(out.float().cpu().numpy(), ref, f"edge {counts} {path}")
 
@@ -135,14 +137,37 @@ def test_empty_input():
     assert out.shape == (0, 128)
 
 
-SAMPLE = np.array([0, 1, 2, 3, 5, 8, 13, 100, 511, 1000, 2047, 3001, 4094, 4095])
+# Per-token bound: the whole-layer tolerance is a norm over all tokens; a
+# localised error (one wrong tile, one wrong token) must also fail. bf16 h and y
+# roundings give a per-token relative error near 3e-3; 4x the layer bound
+# leaves room for the worst of thousands of tokens and none for a wrong one.
+TOKEN_REL_FRO = 2e-2
+
+
+def _expert_block_check(ws, lay, perm, x, idx, W, wl, experts):
+    """h and y of every row of the given experts against the oracle's expert MLP."""
+    m_used = int(perm["off"][-1])
+    h_all = ws[lay.h:lay.h + 2 * m_used * wl.I].view(torch.bfloat16).reshape(m_used, wl.I)
+    y_all = ws[lay.y:lay.y + 2 * m_used * wl.H].view(torch.bfloat16).reshape(m_used, wl.H)
+    V1, V2 = ExpertView(W["w_gate_up"], cache=False), ExpertView(W["w_down"], cache=False)
+    xn = x.float().numpy()
+    for e in experts:
+        r0, c = int(perm["off"][e]), int(perm["cnt"][e])
+        if c == 0:
+            continue
+        a = perm["row_src"][r0:r0 + c]
+        href, yref = O.expert_mlp(xn[a // wl.k].astype(np.float64), V1[e], V2[e], "bf16")
+        assert_bf16_close(h_all[r0:r0 + c].float().cpu().numpy(), href, f"h of expert {e}")
+        assert_bf16_close(y_all[r0:r0 + c].float().cpu().numpy(), yref, f"y of expert {e}")
 
 
 @pytest.mark.parametrize("name", ["prefill", "skewed"])
-def test_full_size_bf16_sampled(name):
+def test_full_size_bf16_every_token(name):
     """Full-size workload in the launch configuration the benchmark times
-    (AUTO path); the oracle computes a sample of tokens one by one, and the
-    permutation is checked in full."""
+    (AUTO path): the oracle computes every token. Permutation bit-exact; the
+    output within the bf16 tolerance as a whole and token by token; the combine
+    bit-exact on the device's own y; h and y element-wise for a block of
+    experts (the first, a middle and the last)."""
     wl = G.WORKLOADS[name]
     seed = G.default_seed(wl)
     x, L, W = device_inputs(wl, seed)
@@ -152,13 +177,24 @@ def test_full_size_bf16_sampled(name):
     idx, w, _ = O.route(L.numpy(), wl.k)
     ws = layer._workspace(wl.T, x.cuda().device)
     assert moe.read_device_status(ws) == 0
-    check_permutation(ws, moe.make_shape(wl.T, wl.H, wl.I, wl.E, wl.k, "bf16", "auto"), idx)
-    toks = np.concatenate([SAMPLE[SAMPLE < wl.T], [wl.T - 1]])
-    ref = oracle_forward_bf16(x, idx, w, W, tokens=toks)
-    assert_bf16_close(out.float().cpu().numpy()[toks], ref, name)
-    # every output row is finite and non-trivial
-    o = out.float()
-    assert torch.isfinite(o).all() and (o.abs().amax(dim=1) > 0).all()
+    shape = moe.make_shape(wl.T, wl.H, wl.I, wl.E, wl.k, "bf16", "auto")
+    lay, perm = check_permutation(ws, shape, idx)
+    check_combine_bit_exact(ws, shape, w, out)
+    _expert_block_check(ws, lay, perm, x, idx, W, wl, [0, wl.E // 2, wl.E - 1])
+    ref = oracle_forward_bf16(x, idx, w, W, cache=False)
+    got = out.float().cpu().numpy()
+    assert_bf16_close(got, ref, name)
+    assert_tokens_close(got, ref, TOKEN_REL_FRO, name)
+
+
+@pytest.mark.parametrize("path", ["prefill", "decode"])
+@pytest.mark.parametrize("name", ["tiny", "decode"])
+def test_combine_bit_exact_given_y(name, path):
+    """The combine alone: fp32 fused multiply-adds in ascending j over the
+    device's expert outputs, rounded once to bf16, bit for bit."""
+    wl = G.WORKLOADS[name]
+    x, idx, w, W, out, ws = _forward(wl, G.default_seed(wl), path)
+    check_combine_bit_exact(ws, moe.make_shape(wl.T, wl.H, wl.I, wl.E, wl.k, "bf16", path), w, out)
 
 
 @pytest.mark.parametrize("name", ["tiny", "decode"])
