@@ -63,3 +63,13 @@ extern "C" moe_status moe_forward_noalloc(const moe_shape* shape, const void* x,
   return moe_forward(shape, x, topk_idx, topk_w, w_gate_up, w_down, sw_gate_up, sw_down, out, scratch,
                      kNoAllocScratchBytes, stream);
 }
+
+// The status word of the last moe_forward_noalloc on the current device: the
+// forward writes device-side errors (a routing index out of range, a bounded
+// wait that gave up) to the first word of its scratch, as moe_forward does to
+// its workspace.
+extern "C" moe_status moe_forward_noalloc_status(void* stream) {
+  void* scratch = scratch_address();
+  if (scratch == nullptr) return MOE_ERR_CUDA;
+  return moe_read_device_status(scratch, stream);
+}

@@ -48,3 +48,39 @@ def test_noalloc_matches_forward_on_two_calls(name, path):
         assert_bf16_close(got.float().cpu().numpy(), ref.float().cpu().numpy(), f"{name} call {call}")
         # same kernels on the same inputs: the results are in fact identical
         assert torch.equal(got, ref)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("wl,path", [
+    (G.Workload("na_fp8_dec", 16, 512, 256, 8, 2, wdtype="e4m3"), "decode"),
+    (G.Workload("na_fp8_pre", 64, 256, 256, 8, 2, wdtype="e4m3"), "prefill"),
+])
+def test_noalloc_fp8_matches_forward_on_two_calls(wl, path):
+    """The e4m3 workspace layouts (x codes and scales, h codes and scales, the
+    fp32 h of the DECODE path) inside the fixed scratch: identical results to
+    moe_forward on a caller workspace, two calls in a row."""
+    shape = moe.make_shape(wl.T, wl.H, wl.I, wl.E, wl.k, "e4m3", path)
+    assert moe.workspace_size(shape) <= 8 << 20
+    W = G.make_weights(wl, 9, device="cuda")
+    for call, seed in enumerate((13, 14)):
+        x, idx, w = _inputs(wl, seed)
+        got = moe.forward_noalloc(x, idx, w, W["w_gate_up"], W["w_down"], W["sw_gate_up"], W["sw_down"], path=path)
+        ref, _ = moe.forward(x, idx, w, W["w_gate_up"], W["w_down"], W["sw_gate_up"], W["sw_down"], path=path)
+        torch.cuda.synchronize()
+        assert torch.equal(got, ref), f"{wl.name} call {call}"
+        assert moe.noalloc_device_status() == 0
+
+
+@pytest.mark.gpu
+def test_noalloc_reports_device_errors():
+    """A routing index out of range reaches the caller through the status
+    word in the scratch; the next good call clears it."""
+    wl = G.Workload("na_bad", 40, 128, 128, 4, 2)
+    W = G.make_weights(wl, 1, device="cuda")
+    x, idx, w = _inputs(wl, 3)
+    bad = idx.clone()
+    bad[3, 1] = 4  # out of range: the permute rejects it without touching memory for it
+    moe.forward_noalloc(x, bad, w, W["w_gate_up"], W["w_down"], path="decode")
+    assert moe.noalloc_device_status() == -7
+    moe.forward_noalloc(x, idx, w, W["w_gate_up"], W["w_down"], path="decode")
+    assert moe.noalloc_device_status() == 0
