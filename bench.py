@@ -1,13 +1,16 @@
 #!/usr/bin/env python
 """Benchmark of the routed MoE expert forward on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--only] [--impl ours|reference]
 
 A step is one pass of the whole hot path on one batch of synthetic input:
 moe_route (router top-k) followed by moe_forward (permute, gate/up with
-SwiGLU, down, combine) of one layer. The default workload is the
-decode-shaped layer (T=16, H=2048, I=1408, E=60, k=4, bf16); --workload picks
-another (tiny, decode, prefill, fp8, skewed, fp8_decode).
+SwiGLU, down, combine) of one layer. The headline workload is the large FP8
+layer (T=4096, H=7168, I=2048, E=256, k=8, e4m3 experts with UE8M0 block
+scales), the largest of the layers; the line's top-level numbers are its own.
+Every other workload (tiny, decode, prefill, skewed, fp8_decode) is measured
+the same way in the same process and reported under "per_config" (--only
+skips them; --workload picks another headline).
 
 Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events
 on the launching stream, with a 256 MiB buffer written between steps (outside
@@ -16,16 +19,17 @@ resident in HBM when a step starts. Multi-GPU (torchrun, one process per GPU)
 runs independent replicas: the layer has no data-path exchange; the elapsed
 time is the max over ranks and the value counts the tokens of all ranks.
 
-The JSON line also carries: the stage breakdown (events recorded by
-moe_forward_timed), the roofline of the dominant kernel (algorithmic bytes or
-FLOPs per launch over its measured duration, against MEASURED_PEAKS.json),
-the end-to-end number through the public API with host buffers (H2D of x and
-logits, D2H of the output inside the timed region), the CPU oracle timed on a
-bounded sample (rank 0, N=1), the number of our kernel launches in the timed
-region, and the SM clocks sampled during it.
+Each workload's entry carries: tokens/s and TFLOP/s, the stage breakdown
+(events recorded by moe_forward_timed), the roofline of the dominant kernel
+(algorithmic bytes or FLOPs per launch over its measured duration, against
+MEASURED_PEAKS.json), the end-to-end number through the public API with host
+buffers (H2D of x and logits, D2H of the output inside the timed region),
+the CPU oracle timed on a bounded sample (rank 0, N=1), the number of our
+kernel launches in the timed region, and the SM clocks sampled while the
+GPU was busy with it.
 
 --impl reference times the CPU oracle (test infrastructure, unmodified) on the
-same workload, a bounded sample of tokens per step, on rank 0 only.
+headline workload, a bounded sample of tokens per step, on rank 0 only.
 """
 from __future__ import annotations
 
@@ -48,18 +52,24 @@ import torch  # noqa: E402
 from mixture_experts_routed_moe_b200 import inputs as G  # noqa: E402
 
 METRIC = "MoE layer tokens/sec and TFLOP/s (% of BF16/FP8 peak or HBM BW) on 1 B200"
-DEFAULT_WORKLOAD = "decode"
+DEFAULT_WORKLOAD = "fp8"
+# measured after the headline, in this order, under "per_config"
+OTHER_WORKLOADS = ["tiny", "decode", "prefill", "skewed", "fp8_decode"]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FLUSH_BYTES = 256 << 20
 
 # DRAM bytes (read + write) per launch of the dominant kernel, from one ncu
-# capture each (profiles/ holds the summaries); a record counts only while its
-# kernel's source file is unchanged (hash of the .cu).
+# capture each; a record counts only while its kernel's source file is
+# unchanged (first 16 hex digits of the .cu file's SHA-256). "scaled" says how
+# a capture of a smaller case was brought to one full launch.
 NCU_TRAFFIC = {
-    ("decode", "decode_gate_up_kernel"): {"bytes": 488557824, "src": "5081ecfb3dbd224e", "from": "profiles/decode_gate_up_kernel__decode.md: full workload"},
-    ("prefill", "grouped_gemm_bf16_kernel<256,true>"): {"bytes": 1199602000, "src": "6c04940ec94b2755", "from": "profiles/grouped_gemm_bf16__prefill.md: full workload"},
-    ("fp8", "grouped_gemm_e4m3_kernel<true>"): {"bytes": 8891190048, "src": "531c17a3a153a8ad", "from": "profiles/grouped_gemm_e4m3__fp8_1024tok_64exp.md: T=1024, E=64 capture x4 (rows and experts scale by 4)"},
-    ("fp8_decode", "decode_e4m3_gate_up_kernel"): {"bytes": 2841453056, "src": "4ecd5f69f521259e", "from": "profiles/decode_e4m3_gate_up_kernel__fp8_2tok_32exp.md: T=2, E=32 capture (14 touched experts) x 94/14 touched"},
+    ("decode", "decode_gate_up_kernel"): {"bytes": 488557824, "src": "5081ecfb3dbd224e", "scaled": None},
+    ("prefill", "grouped_gemm_bf16_kernel<256,true>"): {"bytes": 1199602000, "src": "6c04940ec94b2755",
+                                                         "scaled": None},
+    ("fp8", "grouped_gemm_e4m3_kernel<true>"): {"bytes": 8891190048, "src": "531c17a3a153a8ad",
+                                                "scaled": "T=1024, E=64 capture x4 (rows and experts)"},
+    ("fp8_decode", "decode_e4m3_gate_up_kernel"): {"bytes": 2841453056, "src": "4ecd5f69f521259e",
+                                                   "scaled": "T=2, E=32 capture (14 touched experts) x94/14"},
 }
 
 
@@ -330,7 +340,10 @@ def stage_roofline(wl, path, stage_ms, n_touched, peaks, peak_src):
                    "frac": ach / peaks["hbm_gbs"], "tensor_frac": flops / dur_s / 1e12 / tpeak}
         out.update({"kernel": kern, "stage": names[s], "algorithmic_flops": flops, "algorithmic_bytes": byts})
     rec = NCU_TRAFFIC.get((wl.name, kern))
-    out["traffic"] = rec["bytes"] if rec and rec["src"] == src_hash(src) else None
+    live = rec is not None and rec["src"] == src_hash(src)
+    out["traffic"] = rec["bytes"] if live else None
+    if live and rec["scaled"]:
+        out["traffic_scaled_from"] = rec["scaled"]
     out["peak_from"] = peak_src
     return out
 
@@ -382,10 +395,10 @@ def time_router(moe, wl, seed, xd, flush, stream, K, W, world, peaks):
     return {"ms": ms, "tokens_per_s": wl.T / (ms / 1e3), "launches": K, "roofline": roof}
 
 
-def run_ours(args, world, rank, local):
-    import mixture_experts_routed_moe_b200 as moe
-
-    wl = G.WORKLOADS[args.workload]
+def measure(moe, wl, args, world, rank, local, peaks, peak_src):
+    """One workload: the timed graph steps, the eager stage breakdown, the
+    end-to-end steps with host buffers, the roofline of the dominant kernel and
+    (rank 0, N=1) the CPU oracle on a bounded sample. Returns its JSON dict."""
     seed = G.default_seed(wl)
     dev = torch.device("cuda", local if world > 1 else 0)
     x, logits = G.make_activations(wl, seed)
@@ -429,7 +442,6 @@ def run_ours(args, world, rank, local):
         ev_e[i].record(stream)
     torch.cuda.synchronize()
     barrier(world)
-    clk = clocks.stop()
     step_ms = [ev_s[i].elapsed_time(ev_e[i]) for i in range(K)]
     total_ms = max_over_ranks(sum(step_ms), world)
 
@@ -462,11 +474,11 @@ def run_ours(args, world, rank, local):
         e2e_e[i].record(stream)
     torch.cuda.synchronize()
     barrier(world)
+    clk = clocks.stop()
     e2e_ms = max_over_ranks(sum(e2e_s[i].elapsed_time(e2e_e[i]) for i in range(K)), world)
     if not torch.equal(graph.out, out):
         raise RuntimeError("graph replay and eager forward disagree")
 
-    peaks, peak_src = load_peaks()
     router_line = None
     if args.router and wl.E <= 256:
         router_line = time_router(moe, wl, seed, xd, flush, stream, K, args.warmup, world, peaks)
@@ -476,17 +488,14 @@ def run_ours(args, world, rank, local):
     per_step_launches = (1 + (1 if wl.T <= 256 else 3) + 2 + 1
                          + (2 if path == "decode" and wl.wdtype == "e4m3" else 0))
     tokens = wl.T * K * world
-    value = tokens / (total_ms / 1e3)
     line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
-        "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": wl.wdtype, "data": "synthetic (seeded N(0,1) activations and logits, N(0,0.02) weights)",
-        "config": workload_config(wl, path),
+        "value": tokens / (total_ms / 1e3), "unit": "tokens/s", "ms_per_step": total_ms / K,
         "tflops": wl.flops() * K * world / (total_ms / 1e3) / 1e12,
+        "dtype": wl.wdtype, "config": workload_config(wl, path),
         "stages_ms": {"route": route_ms, "permute": stage_ms[1], "gate_up": stage_ms[2], "down": stage_ms[3],
                       "combine": stage_ms[4], "eager_step": eager_ms},
         "touched_experts": n_touched,
-        "roofline": None,
+        "roofline": stage_roofline(wl, path, {1: stage_ms[2], 2: stage_ms[3]}, n_touched, peaks, peak_src),
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": x.numel() * 2 + logits.numel() * 4, "d2h_bytes_per_step": wl.T * wl.H * 2},
         "gpu_launches": per_step_launches * K,
@@ -494,14 +503,35 @@ def run_ours(args, world, rank, local):
     }
     if router_line is not None:
         line["router"] = router_line
-    # stage indices above: events[0..4] = before permute, after permute, after gate/up, after down, after combine
-    line["roofline"] = stage_roofline(wl, path, {1: stage_ms[2], 2: stage_ms[3]}, n_touched, peaks, peak_src)
+    del graph, layer, W, ws, flush, out, xd, ld
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         n = oracle_sample_tokens(wl)
         rate, per_step, threads, times = oracle_sample_rate(wl, seed, n, steps=1, warmup=0, min_seconds=10.0)
         line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                                 "sample": f"first {n} of {wl.T} tokens, {len(times)} passes "
                                           f"({per_step:.2f} s each, {sum(times):.1f} s in all)"}
+    return line
+
+
+def run_ours(args, world, rank, local):
+    import mixture_experts_routed_moe_b200 as moe
+
+    peaks, peak_src = load_peaks()
+    wl = G.WORKLOADS[args.workload]
+    head = measure(moe, wl, args, world, rank, local, peaks, peak_src)
+    line = {"metric": METRIC, "value": head["value"], "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": wl.wdtype,
+            "data": "synthetic (seeded N(0,1) activations and logits, N(0,0.02) weights)"}
+    line.update({k: v for k, v in head.items() if k not in ("value", "unit", "ms_per_step", "dtype")})
+    if not args.only and wl.name != "custom":
+        per = {}
+        for name in [n for n in [DEFAULT_WORKLOAD] + OTHER_WORKLOADS if n != wl.name]:
+            log(f"measuring {name}")
+            per[name] = measure(moe, G.WORKLOADS[name], args, world, rank, local, peaks, peak_src)
+        line["per_config"] = per
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -514,6 +544,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=list(G.WORKLOADS), default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", action="store_true", help="measure the chosen workload alone (no per_config)")
     ap.add_argument("--router", action="store_true",
                     help="also time the fused router (router GEMM + top-k) on the workload's tokens")
     ap.add_argument("--shape", default=None,
