@@ -19,8 +19,9 @@
 // Warp roles (320 threads, one CTA per SM):
 //   warp 0      TMA producer: A tile [128 x 64] and B tile [N x 64] per stage
 //   warp 1      TMEM allocator and MMA issuer (one thread): 4 MMAs of K=16 per stage
-//   warps 2..9  epilogue: TMEM -> registers -> act(gate)*up / bf16 -> global
-//               memory; two warps per TMEM lane quadrant, half the columns each
+//   warps 2..9  epilogue: TMEM -> registers -> act(gate)*up / bf16 -> a
+//               64-byte-swizzled staging tile in shared memory -> TMA tile
+//               store; two warps per TMEM lane quadrant, half the columns each
 //               (with four, the epilogue took as long as a tile's MMAs)
 // Shared memory holds a 4-stage ring; TMEM holds two accumulators of N fp32
 // columns so the epilogue of one tile overlaps the MMAs of the next.
@@ -44,6 +45,7 @@ struct GemmParams {
   const int* mt_base;  // [E+1] per-expert 128-row tile prefix
   const int* cnt;      // [E]
   int E;
+  int stage_bufs;  // staging tiles per epilogue warp (2 when shared memory allows, else 1)
   int num_kb;             // K / 64
   int n_tiles;            // N blocks per expert
   int b_rows_per_expert;  // rows of one expert's B matrix
@@ -71,22 +73,58 @@ __device__ __forceinline__ bool cluster_tile(int g, int rank, int cs, const int*
   return c->n < NT;
 }
 
+constexpr int kStageBox = 32 * 64;  // one staging tile: 32 rows x 32 bf16 columns (64-byte rows)
+
 template <int kN>
 struct Layout {
   static constexpr int kA = kTileM * kBK * 2;  // 16 KB
   static constexpr int kB = kN * kBK * 2;      // 32 KB for N = 256
   static constexpr int kStage = kA + kB;
   static constexpr int kBarriers = 2 * kStages + 5;
-  static constexpr size_t bytes(int E) {
-    return 1024 /*alignment slack*/ + static_cast<size_t>(kStages) * kStage + kBarriers * 8 + 16 +
+  static constexpr size_t bytes(int E, int bufs) {
+    return 1024 /*alignment slack*/ + static_cast<size_t>(kStages) * kStage +
+           static_cast<size_t>(kEpiWarps) * bufs * kStageBox + kBarriers * 8 + 16 +
            static_cast<size_t>(2 * E + 1) * 4;
   }
 };
 
+// Converts 32 fp32 columns of one row per lane to bf16 and stores the warp's
+// 32 x 32 tile at (x, y) of `map` through the staging buffer `stg` (the TMA
+// store that last read it must be done, which the caller waits for).
+__device__ __forceinline__ void store_box_bf16(const CUtensorMap* map, uint8_t* stg, const uint32_t (&pk)[16],
+                                               bool store, int x, int y, int lane) {
+  const uint32_t sb = smem_u32(stg);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) st_shared_v4(sb + sw64_offset(lane, i), pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+  fence_proxy_async_shared();
+  __syncwarp();
+  if (lane == 0 && store) {
+    tma_store_2d(map, stg, x, y);
+    bulk_commit_group();
+  }
+}
+
+// Staging-buffer rotation of one epilogue warp: wait until the next buffer is
+// free (no TMA store still reads it) and return it.
+__device__ __forceinline__ uint8_t* next_stage(uint8_t* stage0, int bufs, int& buf, int lane) {
+  if (lane == 0) {
+    if (bufs == 2)
+      bulk_wait_group_read<1>();
+    else
+      bulk_wait_group_read<0>();
+  }
+  __syncwarp();
+  uint8_t* stg = stage0 + buf * kStageBox;
+  buf = (buf + 1) % bufs;
+  return stg;
+}
+
 // act(gate) * up for this thread's row: TMEM columns [64*half, 64*half+64) of
-// the gate block and the same of the up block, written as 64 bf16 h values.
+// the gate block and the same of the up block, stored as 64 bf16 h values at
+// columns x0 .. x0+63 of rows y0 .. y0+31 (the warp's rows).
 template <int kAct>
-__device__ __forceinline__ void epilogue_gated(uint32_t tb, int half, bool valid, __nv_bfloat16* dst) {
+__device__ __forceinline__ void epilogue_gated(uint32_t tb, int half, const CUtensorMap* map, uint8_t* stage0,
+                                               int bufs, int& buf, bool store, int x0, int y0, int lane) {
 #pragma unroll 1
   for (int cc = 2 * half; cc < 2 * half + 2; ++cc) {
     uint32_t g[32], u[32];
@@ -98,24 +136,22 @@ __device__ __forceinline__ void epilogue_gated(uint32_t tb, int half, bool valid
     for (int i = 0; i < 16; ++i)
       pk[i] = pack_bf16x2(gated_act_t<kAct>(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i])),
                           gated_act_t<kAct>(__uint_as_float(g[2 * i + 1]), __uint_as_float(u[2 * i + 1])));
-    if (valid) {
-      uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-    }
+    uint8_t* stg = next_stage(stage0, bufs, buf, lane);
+    store_box_bf16(map, stg, pk, store, x0 + (cc - 2 * half) * 32, y0, lane);
   }
 }
 
 template <int kN, bool kSwiGLU>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                             const GemmParams p) {
+                             const __grid_constant__ CUtensorMap tmO, const GemmParams p) {
   using L = Layout<kN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* sA = smem;
   uint8_t* sB = smem + kStages * L::kA;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + kStages * L::kB);
+  uint8_t* sO = sB + kStages * L::kB;  // [8 warps][stage_bufs][kStageBox]
+  uint64_t* full = reinterpret_cast<uint64_t*>(sO + kEpiWarps * p.stage_bufs * kStageBox);
   uint64_t* empty = full + kStages;
   uint64_t* tfull = empty + kStages;  // [2]
   uint64_t* tempty = tfull + 2;       // [2]
@@ -144,6 +180,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&tmA);
     prefetch_tensormap(&tmB);
+    prefetch_tensormap(&tmO);
   }
   if (warp == 1) {
     tmem_alloc(s_tmem, 2 * kN);
@@ -247,7 +284,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // 32*(warp%4) .. +31), each converting half of the tile's columns
     const int quad = warp & 3;
     const int half = (warp - 2) >> 2;
-    const int r = quad * 32 + lane;
+    uint8_t* stage0 = sO + (warp - 2) * p.stage_bufs * kStageBox;
+    int buf = 0;
     int acc = 0;
     uint32_t aph = 0;
     for (int g = first; g < total; g += step) {
@@ -257,15 +295,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * kN);
-      const bool valid = r < c.valid;
-      __nv_bfloat16* dst =
-          p.out + static_cast<size_t>(c.row0 + r) * p.out_ld + static_cast<size_t>(c.n) * p.out_tile_cols;
+      // the warp's 32 rows are stored whole: rows past the expert's count are
+      // pad rows of its own last block, which no later stage reads
+      const int y0 = c.row0 + quad * 32;
+      const int x0 = c.n * p.out_tile_cols + half * (kSwiGLU ? 64 : kN / 2);
       if constexpr (kSwiGLU) {
         // gate columns 0..127, up columns 128..255 of the accumulator
         switch (p.act) {
-          case MOE_ACT_GELU: epilogue_gated<MOE_ACT_GELU>(tb, half, valid, dst); break;
-          case MOE_ACT_RELU: epilogue_gated<MOE_ACT_RELU>(tb, half, valid, dst); break;
-          default: epilogue_gated<MOE_ACT_SILU>(tb, half, valid, dst); break;
+          case MOE_ACT_GELU: epilogue_gated<MOE_ACT_GELU>(tb, half, &tmO, stage0, p.stage_bufs, buf, true, x0, y0, lane); break;
+          case MOE_ACT_RELU: epilogue_gated<MOE_ACT_RELU>(tb, half, &tmO, stage0, p.stage_bufs, buf, true, x0, y0, lane); break;
+          default: epilogue_gated<MOE_ACT_SILU>(tb, half, &tmO, stage0, p.stage_bufs, buf, true, x0, y0, lane); break;
         }
       } else {
         constexpr int kChunks = kN / 32 / 2;  // 32-column chunks per half
@@ -277,11 +316,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-          if (valid) {
-            uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-          }
+          uint8_t* stg = next_stage(stage0, p.stage_bufs, buf, lane);
+          store_box_bf16(&tmO, stg, pk, true, x0 + (cc - half * kChunks) * 32, y0, lane);
         }
       }
       tc_fence_before();
@@ -290,6 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       acc ^= 1;
       if (acc == 0) aph ^= 1;
     }
+    if (lane == 0) bulk_wait_group<0>();  // every store of this warp has landed
   }
 
   __syncthreads();
@@ -300,14 +337,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <int kN, bool kSwiGLU>
-cudaError_t launch_one(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmParams& gp, int grid,
-                       cudaStream_t st) {
-  const size_t smem = Layout<kN>::bytes(gp.E);
+cudaError_t launch_one(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmO, GemmParams gp,
+                       int grid, cudaStream_t st) {
+  gp.stage_bufs = Layout<kN>::bytes(gp.E, 2) <= kSmemLimit ? 2 : 1;
+  const size_t smem = Layout<kN>::bytes(gp.E, gp.stage_bufs);
+  if (smem > kSmemLimit) return cudaErrorInvalidValue;
   static unsigned long long done = 0;
   cudaError_t err = ensure_max_smem(reinterpret_cast<const void*>(grouped_gemm_bf16_kernel<kN, kSwiGLU>), &done);
   if (err != cudaSuccess) return err;
   if (gp.cs == 1) {
-    grouped_gemm_bf16_kernel<kN, kSwiGLU><<<grid, kThreads, smem, st>>>(tmA, tmB, gp);
+    grouped_gemm_bf16_kernel<kN, kSwiGLU><<<grid, kThreads, smem, st>>>(tmA, tmB, tmO, gp);
     return cudaGetLastError();
   }
   // every cluster of the persistent grid must be resident at once: with an
@@ -327,7 +366,7 @@ cudaError_t launch_one(const CUtensorMap& tmA, const CUtensorMap& tmB, const Gem
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, grouped_gemm_bf16_kernel<kN, kSwiGLU>, tmA, tmB, gp);
+  return cudaLaunchKernelEx(&cfg, grouped_gemm_bf16_kernel<kN, kSwiGLU>, tmA, tmB, tmO, gp);
 }
 
 }  // namespace
@@ -361,11 +400,13 @@ cudaError_t launch_gemm_bf16(const moe_shape* s, const Plan& p, const void* w_ga
   gp.act = s->act;
   // every tile count is bounded by the row capacity
   const int max_mtiles = static_cast<int>(p.m_rows / kTileM);
-  CUtensorMap tmA, tmB;
+  CUtensorMap tmA, tmB, tmO;
   if (which == 0) {
     if (!encode_tensor_map_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws + p.xa, H, p.m_rows, kBK, kTileM) ||
         !encode_tensor_map_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w_gate_up, H,
-                              static_cast<uint64_t>(E) * 2 * I, kBK, 128))
+                              static_cast<uint64_t>(E) * 2 * I, kBK, 128) ||
+        !encode_tensor_map_2d(&tmO, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws + p.h, I, p.m_rows, 32, 32,
+                              CU_TENSOR_MAP_SWIZZLE_64B))
       return cudaErrorInvalidValue;
     gp.num_kb = H / kBK;
     gp.n_tiles = I / 128;
@@ -378,11 +419,13 @@ cudaError_t launch_gemm_bf16(const moe_shape* s, const Plan& p, const void* w_ga
     gp.cs = gate_up_cluster_size(s, gp.n_tiles, num_sms);
     const int groups = max_mtiles * ((gp.n_tiles + gp.cs - 1) / gp.cs);
     const int grid = gp.cs * std::max(1, std::min(num_sms / gp.cs, groups));
-    return launch_one<256, true>(tmA, tmB, gp, grid, st);
+    return launch_one<256, true>(tmA, tmB, tmO, gp, grid, st);
   }
   if (!encode_tensor_map_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws + p.h, I, p.m_rows, kBK, kTileM) ||
       !encode_tensor_map_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w_down, I, static_cast<uint64_t>(E) * H, kBK,
-                            128))
+                            128) ||
+      !encode_tensor_map_2d(&tmO, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws + p.y, H, p.m_rows, 32, 32,
+                            CU_TENSOR_MAP_SWIZZLE_64B))
     return cudaErrorInvalidValue;
   gp.num_kb = I / kBK;
   gp.b_rows_per_expert = H;
@@ -394,7 +437,7 @@ cudaError_t launch_gemm_bf16(const moe_shape* s, const Plan& p, const void* w_ga
   gp.b_tile_stride = 128;
   gp.out_tile_cols = 128;
   const int grid = std::max(1, std::min(num_sms, max_mtiles * gp.n_tiles));
-  return launch_one<128, false>(tmA, tmB, gp, grid, st);
+  return launch_one<128, false>(tmA, tmB, tmO, gp, grid, st);
 }
 
 }  // namespace moe

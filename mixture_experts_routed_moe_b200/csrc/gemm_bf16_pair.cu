@@ -14,6 +14,10 @@
 // barriers of both CTAs. Each CTA's TMEM holds its 128 rows of the
 // accumulator (two 256-column buffers), which its own epilogue drains; the
 // peer's epilogue releases a buffer by arriving on the leader's barrier.
+// The epilogue converts 32 columns at a time to bf16, writes them into a
+// 64-byte-swizzled staging tile in shared memory (two per warp, so one fills
+// while the other is read) and stores it with a TMA tile store; the release of
+// the accumulator therefore never waits for global stores to drain.
 //
 // Tiles pair up consecutive 128-row blocks of one expert (an expert with an
 // odd count pairs its last block with rows the peer computes and discards).
@@ -34,9 +38,13 @@ constexpr int kB = 128 * kBK * 2;     // this CTA's half of B: 16 KB
 constexpr int kStage = kA + kB;
 constexpr int kN = 256;  // MMA N: both halves of B
 constexpr int kBarriers = 2 * kStages + 5;
+constexpr int kEpiWarps = 4;
+constexpr int kStageBox = 32 * 64;  // one staging tile: 32 rows x 32 bf16 columns (64-byte rows)
+constexpr int kStaging = kEpiWarps * 2 * kStageBox;
 
 size_t pair_smem_bytes(int E) {
-  return 1024 + static_cast<size_t>(kStages) * kStage + kBarriers * 8 + 16 + static_cast<size_t>(3 * E + 2) * 4;
+  return 1024 + static_cast<size_t>(kStages) * kStage + kStaging + kBarriers * 8 + 16 +
+         static_cast<size_t>(3 * E + 2) * 4;
 }
 
 struct PairParams {
@@ -76,12 +84,13 @@ __device__ __forceinline__ PairCoord pair_coord(int tile, const int* s_pt, const
 
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                                  const PairParams p) {
+                                  const __grid_constant__ CUtensorMap tmY, const PairParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* sA = smem;
   uint8_t* sB = smem + kStages * kA;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + kStages * kB);  // used in the leader
+  uint8_t* sY = sB + kStages * kB;                                    // [4 warps][2][kStageBox]
+  uint64_t* full = reinterpret_cast<uint64_t*>(sY + kStaging);  // used in the leader
   uint64_t* empty = full + kStages;
   uint64_t* tfull = empty + kStages;  // [2]
   uint64_t* tempty = tfull + 2;       // [2] used in the leader: 4 warps of each CTA arrive
@@ -116,6 +125,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&tmA);
     prefetch_tensormap(&tmB);
+    prefetch_tensormap(&tmY);
   }
   if (warp == 1) {
     tmem_alloc_pair(s_tmem, 2 * kN);
@@ -207,7 +217,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ---------------- epilogue (both CTAs, own 128 rows) ----------------
     const int quad = warp & 3;
-    const int r = quad * 32 + lane;
+    uint8_t* stage0 = sY + (warp - 2) * 2 * kStageBox;
+    int buf = 0;
     int acc = 0;
     uint32_t aph = 0;
     for (int tile = cluster; tile < total; tile += nclusters) {
@@ -216,22 +227,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * kN);
-      const bool valid = r < c.valid;
-      __nv_bfloat16* dst =
-          p.out + static_cast<size_t>(c.row0 + r) * p.out_ld + static_cast<size_t>(c.n) * p.out_tile_cols;
+      // a block past the end of its expert (the peer's half of an odd last
+      // pair) aliases the next expert's rows: never stored. Pad rows inside a
+      // block hold garbage that no later stage reads, and are stored with it.
+      const bool store = c.valid > 0;
 #pragma unroll 1
       for (int cc = 0; cc < kN / 32; ++cc) {
         uint32_t v[32];
         tmem_ld32(tb + cc * 32, v);
         tmem_ld_wait();
-        uint32_t pk[16];
+        uint8_t* stg = stage0 + buf * kStageBox;
+        if (lane == 0) bulk_wait_group_read<1>();  // the store that last read this buffer is done with it
+        __syncwarp();
+        const uint32_t sb = smem_u32(stg);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-        if (valid) {
-          uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+        for (int i = 0; i < 4; ++i)
+          st_shared_v4(sb + sw64_offset(lane, i), pack_bf16x2(__uint_as_float(v[8 * i]), __uint_as_float(v[8 * i + 1])),
+                       pack_bf16x2(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3])),
+                       pack_bf16x2(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5])),
+                       pack_bf16x2(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7])));
+        fence_proxy_async_shared();
+        __syncwarp();
+        if (lane == 0 && store) {
+          tma_store_2d(&tmY, stg, c.n * p.out_tile_cols + cc * 32, c.row0 + quad * 32);
+          bulk_commit_group();
         }
+        buf ^= 1;
       }
       tc_fence_before();
       __syncwarp();
@@ -239,6 +260,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       acc ^= 1;
       if (acc == 0) aph ^= 1;
     }
+    if (lane == 0) bulk_wait_group<0>();  // every store of this warp has landed
   }
 
   __syncthreads();
@@ -249,8 +271,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-cudaError_t launch_pair(const CUtensorMap& tmA, const CUtensorMap& tmB, const PairParams& pp, int nclusters,
-                        cudaStream_t st) {
+cudaError_t launch_pair(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmY, const PairParams& pp,
+                        int nclusters, cudaStream_t st) {
   static unsigned long long done = 0;
   cudaError_t err = ensure_max_smem(reinterpret_cast<const void*>(grouped_gemm_bf16_pair_kernel), &done);
   if (err != cudaSuccess) return err;
@@ -271,7 +293,7 @@ cudaError_t launch_pair(const CUtensorMap& tmA, const CUtensorMap& tmB, const Pa
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, grouped_gemm_bf16_pair_kernel, tmA, tmB, pp);
+  return cudaLaunchKernelEx(&cfg, grouped_gemm_bf16_pair_kernel, tmA, tmB, tmY, pp);
 }
 
 }  // namespace
@@ -289,12 +311,15 @@ cudaError_t launch_gemm_bf16_pair(const moe_shape* s, const Plan& p, const void*
   pp.timeout_ns = wait_limit_ns();
   // upper bound of the pair-tile count: every expert's pairs fit in (row blocks + E) / 2 + E
   const int max_pairs = static_cast<int>(p.m_rows / kTileM) / 2 + E;
-  CUtensorMap tmA, tmB;
+  CUtensorMap tmA, tmB, tmY;
   if (which != 1) return cudaErrorNotSupported;
   if (H % 256 != 0) return cudaErrorNotSupported;
+  if (pair_smem_bytes(E) > kSmemLimit) return cudaErrorInvalidValue;
   if (!encode_tensor_map_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws + p.h, I, p.m_rows, kBK, kTileM) ||
       !encode_tensor_map_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w_down, I, static_cast<uint64_t>(E) * H, kBK,
-                            128))
+                            128) ||
+      !encode_tensor_map_2d(&tmY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws + p.y, H, p.m_rows, 32, 32,
+                            CU_TENSOR_MAP_SWIZZLE_64B))
     return cudaErrorInvalidValue;
   pp.num_kb = I / kBK;
   pp.n_tiles = H / 256;
@@ -305,7 +330,7 @@ cudaError_t launch_gemm_bf16_pair(const moe_shape* s, const Plan& p, const void*
   pp.out_ld = H;
   pp.out_tile_cols = 256;
   const int nclusters = std::max(1, std::min(num_sms / 2, max_pairs * pp.n_tiles));
-  return launch_pair(tmA, tmB, pp, nclusters, st);
+  return launch_pair(tmA, tmB, tmY, pp, nclusters, st);
 }
 
 }  // namespace moe

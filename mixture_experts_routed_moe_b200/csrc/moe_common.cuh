@@ -114,6 +114,46 @@ __device__ __forceinline__ uint64_t l2_policy_evict_first() {
   return pol;
 }
 
+// TMA tile store from this CTA's shared memory to global memory, tracked as a
+// bulk async group of the issuing thread. The shared-memory source must have
+// been written before a fence_proxy_async_shared() by the writing threads.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* smem_src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(smem_src)), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until at most N of this thread's bulk groups still read shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_group_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+// Wait until at most N of this thread's bulk groups are still in flight (writes included).
+template <int N>
+__device__ __forceinline__ void bulk_wait_group() {
+  asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
+}
+// Makes this thread's generic-proxy shared-memory writes visible to the async
+// proxy (a following TMA store reads them).
+__device__ __forceinline__ void fence_proxy_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+// Byte offset of 16-byte chunk `chunk` (0..7) of row `row` inside a tile of
+// 128-byte rows laid out with the 128-byte TMA swizzle (tile base 1024-byte
+// aligned): the chunk index is XORed with the row's position in its 8-row atom.
+__device__ __forceinline__ uint32_t sw128_offset(int row, int chunk) {
+  return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
+}
+// The same for 64-byte rows under the 64-byte swizzle (tile base 512-byte
+// aligned): chunk (0..3) XOR bits 1..2 of the row.
+__device__ __forceinline__ uint32_t sw64_offset(int row, int chunk) {
+  return static_cast<uint32_t>(row * 64 + ((chunk ^ ((row >> 1) & 3)) << 4));
+}
+__device__ __forceinline__ void st_shared_v4(uint32_t saddr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(saddr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -325,6 +365,19 @@ __device__ __forceinline__ float gated_act(int act, float g, float u) {
   else
     a = g / (1.0f + __expf(-g));
   return a * u;
+}
+
+// (a0, a1) = (b0 * s + a0, b1 * s + a1): two fp32 fused multiply-adds, round to
+// nearest, in one packed f32x2 instruction (each lane bit-identical to fmaf).
+__device__ __forceinline__ void ffma2(float& a0, float& a1, float b0, float b1, float s) {
+  asm("{\n\t.reg .b64 acc, mul, sc;\n\t"
+      "mov.b64 acc, {%0, %1};\n\t"
+      "mov.b64 mul, {%2, %3};\n\t"
+      "mov.b64 sc, {%4, %4};\n\t"
+      "fma.rn.f32x2 acc, mul, sc, acc;\n\t"
+      "mov.b64 {%0, %1}, acc;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "f"(b0), "f"(b1), "f"(s));
 }
 
 // Streaming 16-byte load that does not allocate in L1.
