@@ -19,7 +19,14 @@
 // allocator and MMA issuer, warps 2..9 promotion + epilogue. Warps w and w+4
 // share TMEM lane quadrant w%4 (rows); warp group 2..5 takes the first half of
 // each 128-column block pair, 6..9 the second. Tiles and their order are those
-// of the bf16 kernel (tile_sched.cuh).
+// of the bf16 kernel (tile_sched.cuh), handed out dynamically: the producer
+// takes the next tile number from a counter as its CTA frees up, so CTAs
+// running at the same time work on consecutive tiles (the row blocks of one
+// expert and column block, which share the weight tile through L2) and the
+// load evens out across SMs. A tile's results (h codes, or y) leave
+// through 64-byte-swizzled staging tiles in shared memory and TMA tile stores,
+// so the tile end issues a few shared-memory stores instead of scattered
+// 16-byte global stores, one row per lane.
 #include "moe_common.cuh"
 #include "moe_internal.h"
 #include "tile_sched.cuh"
@@ -34,12 +41,17 @@ constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kA = kTileM * kBK;  // 16 KB
 constexpr int kB = 256 * kBK;     // 32 KB
 constexpr int kStage = kA + kB;
-constexpr int kBarriers = 2 * kStages + 5;
+constexpr int kBarriers = 2 * kStages + 5 + 2 * kTileRing;
+constexpr int kStageBox = 32 * 64;  // one staging tile: 32 rows of 64 bytes
+constexpr int kStaging = kEpiWarps * 2 * kStageBox;
 
-size_t smem_bytes(int E) {
-  return 1024 + static_cast<size_t>(kStages) * kStage + kBarriers * 8 + 16 + 2 * kTileM * 4 +
-         static_cast<size_t>(2 * E + 1) * 4;
-}
+// The expert tile prefix and counts live in shared memory when they fit next
+// to the ring and the staging tiles, else the kernel reads them from global
+// memory (through L1).
+constexpr size_t kFixedSmem =
+    1024 + static_cast<size_t>(kStages) * kStage + kStaging + kBarriers * 8 + 16 + 2 * kTileM * 4 + kTileRing * 4;
+bool sched_in_smem(int E) { return kFixedSmem + static_cast<size_t>(2 * E + 1) * 4 <= kSmemLimit; }
+size_t smem_bytes(int E) { return kFixedSmem + (sched_in_smem(E) ? static_cast<size_t>(2 * E + 1) * 4 : 0); }
 
 struct Fp8Params {
   const int* mt_base;
@@ -52,10 +64,10 @@ struct Fp8Params {
   int b_second_offset;    // B rows from the first 128-row half to the second
   const float* a_scale;   // [m_rows, num_kb]
   const uint8_t* w_scale; // [E, b_rows_per_expert/128, num_kb]
-  uint8_t* hq;            // gate/up: e4m3 h [m_rows, I]
   float* hs;              // gate/up: h scales [m_rows, I/128]
-  __nv_bfloat16* y;       // down: [m_rows, H]
   int out_ld;             // I (gate/up) or H (down)
+  int sched_smem;         // 1: expert prefix and counts copied to shared memory
+  int* tile_counter;      // next tile to hand out (zero at launch)
   int act;                // gate activation (moe_activation)
   int* dev_status;
   unsigned long long timeout_ns;
@@ -63,13 +75,40 @@ struct Fp8Params {
 
 __device__ __forceinline__ void epi_bar_sync() { asm volatile("bar.sync 1, %0;" ::"n"(32 * kEpiWarps) : "memory"); }
 
+// Staging-buffer rotation of one epilogue warp (two buffers): wait until the
+// TMA store that last read the next buffer is done with it.
+__device__ __forceinline__ uint8_t* next_stage(uint8_t* stage0, int& buf, int lane) {
+  if (lane == 0) bulk_wait_group_read<1>();
+  __syncwarp();
+  uint8_t* stg = stage0 + buf * kStageBox;
+  buf ^= 1;
+  return stg;
+}
+
+// Stores the warp's 32 rows x 64 bytes (4 x 16 bytes per lane, one row per
+// lane) at (x, y) of `map` through staging buffer `stg`.
+__device__ __forceinline__ void store_box(const CUtensorMap* map, uint8_t* stg, const uint32_t (&w)[16], int x, int y,
+                                          int lane) {
+  const uint32_t sb = smem_u32(stg);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) st_shared_v4(sb + sw64_offset(lane, i), w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+  fence_proxy_async_shared();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(map, stg, x, y);
+    bulk_commit_group();
+  }
+}
+
 // End of a gate/up tile for one thread's row: h = act(gate) * up on its 64
 // columns, the row's amax over the 128-column group (this warp's half and the
 // partner warp's, exchanged through shared memory), then the 1x128 e4m3 codes
-// and the group scale. The activation is fixed at compile time.
+// (stored with the warp's other rows at (x0, y0) of the h-code map) and the
+// group scale. The activation is fixed at compile time.
 template <int kAct>
 __device__ __forceinline__ void finish_gate_up(float (&acc)[128], float* s_amax, int hf, int r, bool valid,
-                                               uint8_t* hrow, float* hs) {
+                                               const CUtensorMap* map, uint8_t* stg, int x0, int y0, int lane,
+                                               float* hs) {
   float amax = 0.f;
 #pragma unroll
   for (int i = 0; i < 64; ++i) {
@@ -81,45 +120,50 @@ __device__ __forceinline__ void finish_gate_up(float (&acc)[128], float* s_amax,
   amax = fmaxf(s_amax[r], s_amax[kTileM + r]);
   epi_bar_sync();
   const float sc = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
-  if (valid) {
-    uint32_t w[16];
+  uint32_t w[16];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(__fdiv_rn(acc[4 * i], sc), __fdiv_rn(acc[4 * i + 1], sc)),
-                                                   __NV_SATFINITE, __NV_E4M3);
-      const uint32_t hi = __nv_cvt_float2_to_fp8x2(
-          make_float2(__fdiv_rn(acc[4 * i + 2], sc), __fdiv_rn(acc[4 * i + 3], sc)), __NV_SATFINITE, __NV_E4M3);
-      w[i] = lo | (hi << 16);
-    }
-    uint4* dst = reinterpret_cast<uint4*>(hrow);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
-    if (hf == 0) *hs = sc;
+  for (int i = 0; i < 16; ++i) {
+    const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(__fdiv_rn(acc[4 * i], sc), __fdiv_rn(acc[4 * i + 1], sc)),
+                                                 __NV_SATFINITE, __NV_E4M3);
+    const uint32_t hi = __nv_cvt_float2_to_fp8x2(
+        make_float2(__fdiv_rn(acc[4 * i + 2], sc), __fdiv_rn(acc[4 * i + 3], sc)), __NV_SATFINITE, __NV_E4M3);
+    w[i] = lo | (hi << 16);
   }
+  // pad rows of the expert's last block are stored too (nothing reads them)
+  store_box(map, stg, w, x0, y0, lane);
+  if (valid && hf == 0) *hs = sc;
 }
 
 template <bool kGateUp>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_e4m3_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                             const Fp8Params p) {
+                             const __grid_constant__ CUtensorMap tmO, const Fp8Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* sA = smem;
   uint8_t* sB = smem + kStages * kA;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + kStages * kB);
+  uint8_t* sO = sB + kStages * kB;  // [8 warps][2][kStageBox]
+  uint64_t* full = reinterpret_cast<uint64_t*>(sO + kStaging);
   uint64_t* empty = full + kStages;
   uint64_t* pfull = empty + kStages;  // [2] partial accumulator ready
   uint64_t* pempty = pfull + 2;       // [2] partial accumulator consumed
   uint64_t* drain = pempty + 2;
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain + 1);
+  TileRing ring;
+  ring.full = drain + 1;                // [kTileRing]
+  ring.empty = ring.full + kTileRing;   // [kTileRing]
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(ring.empty + kTileRing);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
   float* s_amax = reinterpret_cast<float*>(s_tmem + 4);  // [2][128]
-  int* s_mt = reinterpret_cast<int*>(s_amax + 2 * kTileM);
-  int* s_cnt = s_mt + p.E + 1;
+  ring.ids = reinterpret_cast<int*>(s_amax + 2 * kTileM);  // [kTileRing]
+  int* s_sched = ring.ids + kTileRing;
+  const int* s_mt = p.sched_smem ? s_sched : p.mt_base;
+  const int* s_cnt = p.sched_smem ? s_sched + p.E + 1 : p.cnt;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int i = threadIdx.x; i <= p.E; i += kThreads) s_mt[i] = p.mt_base[i];
-  for (int i = threadIdx.x; i < p.E; i += kThreads) s_cnt[i] = p.cnt[i];
+  if (p.sched_smem) {
+    for (int i = threadIdx.x; i <= p.E; i += kThreads) s_sched[i] = p.mt_base[i];
+    for (int i = threadIdx.x; i < p.E; i += kThreads) s_sched[p.E + 1 + i] = p.cnt[i];
+  }
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
@@ -129,6 +173,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&pfull[b], 1);
       mbar_init(&pempty[b], kEpiWarps);
     }
+    for (int i = 0; i < kTileRing; ++i) {
+      mbar_init(&ring.full[i], 1);
+      mbar_init(&ring.empty[i], 1 + kEpiWarps);  // the MMA issuer and every epilogue warp read each tile
+    }
     mbar_init(drain, 1);
     *s_abort = 0;
     fence_mbarrier_init();
@@ -136,6 +184,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&tmA);
     prefetch_tensormap(&tmB);
+    prefetch_tensormap(&tmO);
   }
   if (warp == 1) {
     tmem_alloc(s_tmem, 512);
@@ -159,7 +208,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t ph = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+      for (int seq = 0; ok; ++seq) {
+        const int tile = tiles_publish(ring, seq, p.tile_counter, total, s_abort, p.dev_status, p.timeout_ns);
+        if (tile < 0) break;
         const TileCoord c = tile_coord(tile, s_mt, s_cnt, p.E, NT);
         const int brow = c.e * p.b_rows_per_expert + c.n * p.b_tile_stride;
         for (int kb = 0; kb < KB; ++kb) {
@@ -195,7 +246,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0, pb = 0;
       uint32_t ph = 0, pph = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+      for (int seq = 0; ok; ++seq) {
+        if (tiles_take(ring, seq, s_abort, p.dev_status, p.timeout_ns) < 0) break;
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait_bounded(&full[stage], ph, s_abort, p.dev_status, p.timeout_ns) ||
               !mbar_wait_bounded(&pempty[pb], pph ^ 1, s_abort, p.dev_status, p.timeout_ns)) {
@@ -229,10 +281,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int hf = (warp - 2) >> 2;  // 0: warps 2..5, 1: warps 6..9
     const int r = quad * 32 + lane;
     const int wrows = p.b_rows_per_expert / 128;  // weight scale rows per expert
+    uint8_t* stage0 = sO + (warp - 2) * 2 * kStageBox;
+    int buf = 0;
     int pb = 0;
     uint32_t pph = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+    for (int seq = 0; ok; ++seq) {
+      const int tile = tiles_take_warp(ring, seq, lane, s_abort, p.dev_status, p.timeout_ns);
+      if (tile < 0) break;
       const TileCoord c = tile_coord(tile, s_mt, s_cnt, p.E, NT);
       const int row = c.row0 + r;
       // weight scale rows of the two 128-column halves this thread promotes
@@ -281,7 +337,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int qq = q + j;
             const float sc = (kGateUp && qq >= 4) ? sc1 : sc0;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) acc[16 * qq + i] = fmaf(__uint_as_float(v[j][i]), sc, acc[16 * qq + i]);
+            for (int i = 0; i < 16; i += 2)
+              ffma2(acc[16 * qq + i], acc[16 * qq + i + 1], __uint_as_float(v[j][i]), __uint_as_float(v[j][i + 1]), sc);
           }
         }
         tc_fence_before();
@@ -295,26 +352,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       // enter the named barrier below without it
       if (__any_sync(0xffffffffu, *s_abort != 0)) break;
       const bool valid = r < c.valid;
+      const int y0 = c.row0 + quad * 32;
       if constexpr (kGateUp) {
         // h for columns n*128 + 64hf + i, i < 64: acc[i] is the gate, acc[64+i] the up projection
-        uint8_t* hrow = p.hq + static_cast<size_t>(row) * p.out_ld + c.n * 128 + hf * 64;
         float* hs = p.hs + static_cast<size_t>(row) * (p.out_ld / 128) + c.n;
+        uint8_t* stg = next_stage(stage0, buf, lane);
+        const int x0 = c.n * 128 + hf * 64;
         switch (p.act) {
-          case MOE_ACT_GELU: finish_gate_up<MOE_ACT_GELU>(acc, s_amax, hf, r, valid, hrow, hs); break;
-          case MOE_ACT_RELU: finish_gate_up<MOE_ACT_RELU>(acc, s_amax, hf, r, valid, hrow, hs); break;
-          default: finish_gate_up<MOE_ACT_SILU>(acc, s_amax, hf, r, valid, hrow, hs); break;
+          case MOE_ACT_GELU: finish_gate_up<MOE_ACT_GELU>(acc, s_amax, hf, r, valid, &tmO, stg, x0, y0, lane, hs); break;
+          case MOE_ACT_RELU: finish_gate_up<MOE_ACT_RELU>(acc, s_amax, hf, r, valid, &tmO, stg, x0, y0, lane, hs); break;
+          default: finish_gate_up<MOE_ACT_SILU>(acc, s_amax, hf, r, valid, &tmO, stg, x0, y0, lane, hs); break;
         }
       } else {
-        if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(p.y + static_cast<size_t>(row) * p.out_ld + c.n * 256 + hf * 128);
+        // y columns n*256 + 128hf + 32q .. +31, one staging tile each
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            dst[i] = make_uint4(pack_bf16x2(acc[8 * i], acc[8 * i + 1]), pack_bf16x2(acc[8 * i + 2], acc[8 * i + 3]),
-                                pack_bf16x2(acc[8 * i + 4], acc[8 * i + 5]),
-                                pack_bf16x2(acc[8 * i + 6], acc[8 * i + 7]));
+        for (int q = 0; q < 4; ++q) {
+          uint32_t w[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) w[i] = pack_bf16x2(acc[32 * q + 2 * i], acc[32 * q + 2 * i + 1]);
+          uint8_t* stg = next_stage(stage0, buf, lane);
+          store_box(&tmO, stg, w, c.n * 256 + hf * 128 + q * 32, y0, lane);
         }
       }
     }
+    if (lane == 0) bulk_wait_group<0>();  // every store of this warp has landed
   }
 
   __syncthreads();
@@ -325,13 +386,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <bool kGateUp>
-cudaError_t launch_one(const CUtensorMap& tmA, const CUtensorMap& tmB, const Fp8Params& fp, int grid,
+cudaError_t launch_one(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmO, Fp8Params fp, int grid,
                        cudaStream_t st) {
+  fp.sched_smem = sched_in_smem(fp.E) ? 1 : 0;
   const size_t smem = smem_bytes(fp.E);
+  if (smem > kSmemLimit) return cudaErrorInvalidValue;
   static unsigned long long done = 0;
   cudaError_t err = ensure_max_smem(reinterpret_cast<const void*>(grouped_gemm_e4m3_kernel<kGateUp>), &done);
   if (err != cudaSuccess) return err;
-  grouped_gemm_e4m3_kernel<kGateUp><<<grid, kThreads, smem, st>>>(tmA, tmB, fp);
+  grouped_gemm_e4m3_kernel<kGateUp><<<grid, kThreads, smem, st>>>(tmA, tmB, tmO, fp);
   return cudaGetLastError();
 }
 
@@ -352,12 +415,16 @@ cudaError_t launch_gemm_e4m3(const moe_shape* s, const Plan& p, const void* /*x*
   fp.dev_status = reinterpret_cast<int*>(ws + p.status);
   fp.timeout_ns = wait_limit_ns();
   fp.act = s->act;
+  // one tile counter per launch, zeroed with the status word by the permute stage
+  fp.tile_counter = reinterpret_cast<int*>(ws + p.status) + kStatusTileCounter + which;
   const int max_mtiles = static_cast<int>(p.m_rows / kTileM);
-  CUtensorMap tmA, tmB;
+  CUtensorMap tmA, tmB, tmO;
   if (which == 0) {
     if (!encode_tensor_map_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ws + p.xa, H, p.m_rows, kBK, kTileM) ||
         !encode_tensor_map_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w_gate_up, H, static_cast<uint64_t>(E) * 2 * I,
-                              kBK, 128))
+                              kBK, 128) ||
+        !encode_tensor_map_2d(&tmO, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ws + p.h, I, p.m_rows, 64, 32,
+                              CU_TENSOR_MAP_SWIZZLE_64B))
       return cudaErrorInvalidValue;
     fp.num_kb = H / kBK;
     fp.n_tiles = I / 128;
@@ -366,16 +433,17 @@ cudaError_t launch_gemm_e4m3(const moe_shape* s, const Plan& p, const void* /*x*
     fp.b_second_offset = I;
     fp.a_scale = reinterpret_cast<const float*>(ws + p.xs);
     fp.w_scale = sw_gate_up;
-    fp.hq = ws + p.h;
     fp.hs = reinterpret_cast<float*>(ws + p.hs);
     fp.out_ld = I;
     const int grid = std::max(1, std::min(num_sms, max_mtiles * fp.n_tiles));
-    return launch_one<true>(tmA, tmB, fp, grid, st);
+    return launch_one<true>(tmA, tmB, tmO, fp, grid, st);
   }
   if (H % 256 != 0) return cudaErrorNotSupported;  // the down tile spans two 128-column scale blocks
   if (!encode_tensor_map_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ws + p.h, I, p.m_rows, kBK, kTileM) ||
       !encode_tensor_map_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w_down, I, static_cast<uint64_t>(E) * H, kBK,
-                            128))
+                            128) ||
+      !encode_tensor_map_2d(&tmO, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws + p.y, H, p.m_rows, 32, 32,
+                            CU_TENSOR_MAP_SWIZZLE_64B))
     return cudaErrorInvalidValue;
   fp.num_kb = I / kBK;
   fp.n_tiles = H / 256;
@@ -384,10 +452,9 @@ cudaError_t launch_gemm_e4m3(const moe_shape* s, const Plan& p, const void* /*x*
   fp.b_second_offset = 128;
   fp.a_scale = reinterpret_cast<const float*>(ws + p.hs);
   fp.w_scale = sw_down;
-  fp.y = reinterpret_cast<__nv_bfloat16*>(ws + p.y);
   fp.out_ld = H;
   const int grid = std::max(1, std::min(num_sms, max_mtiles * fp.n_tiles));
-  return launch_one<false>(tmA, tmB, fp, grid, st);
+  return launch_one<false>(tmA, tmB, tmO, fp, grid, st);
 }
 
 }  // namespace moe

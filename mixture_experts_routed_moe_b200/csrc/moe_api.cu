@@ -48,7 +48,8 @@ std::atomic<int> g_sm_count[kMaxDevices];
 }  // namespace
 
 bool encode_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, size_t elem_bytes, const void* base,
-                          uint64_t inner, uint64_t outer, uint32_t box_inner, uint32_t box_outer) {
+                          uint64_t inner, uint64_t outer, uint32_t box_inner, uint32_t box_outer,
+                          CUtensorMapSwizzle swizzle) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
   const cuuint64_t dims[2] = {inner, outer};
@@ -56,8 +57,7 @@ bool encode_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, size_t el
   const cuuint32_t box[2] = {box_inner, box_outer};
   const cuuint32_t estr[2] = {1, 1};
   return fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+            swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 int device_sm_count() {
@@ -92,8 +92,10 @@ bool validate_shape(const moe_shape* s) {
   if (s->T < 0 || s->H < 128 || s->I < 128 || s->H % 128 != 0 || s->I % 128 != 0) return false;
   if (s->H > 65536 || s->I > 65536) return false;
   if (s->E < 1 || s->E > 1024 || s->k < 1 || s->k > s->E) return false;
-  if (s->wdtype != MOE_DT_BF16 && s->wdtype != MOE_DT_E4M3) return false;
-  if (s->path != MOE_PATH_AUTO && s->path != MOE_PATH_PREFILL && s->path != MOE_PATH_DECODE) return false;
+  if (s->wdtype != MOE_DT_BF16 && s->wdtype != MOE_DT_E4M3 && s->wdtype != MOE_DT_E2M1) return false;
+  if (s->path != MOE_PATH_AUTO && s->path != MOE_PATH_PREFILL && s->path != MOE_PATH_DECODE &&
+      s->path != MOE_PATH_FUSED)
+    return false;
   if (s->act != MOE_ACT_SILU && s->act != MOE_ACT_GELU && s->act != MOE_ACT_RELU) return false;
   const long long A = static_cast<long long>(s->T) * s->k;
   const long long rows = A + static_cast<long long>(std::min<long long>(s->E, A)) * (kTileM - 1) + kTileM;
@@ -116,7 +118,8 @@ bool make_plan(const moe_shape* s, Plan* p) {
   const long long A = T * k;
   const bool fp8 = s->wdtype == MOE_DT_E4M3;
   p->path = resolve_path(s);
-  p->bm = (p->path == MOE_PATH_DECODE) ? 1 : kTileM;
+  const bool streaming = p->path == MOE_PATH_DECODE || p->path == MOE_PATH_FUSED;  // tile size 1, x read in place
+  p->bm = streaming ? 1 : kTileM;
   if (p->bm == 1) {
     p->m_rows = A;
   } else {
@@ -142,16 +145,17 @@ bool make_plan(const moe_shape* s, Plan* p) {
   p->local_rank = take(std::max<long long>(A, 1) * 4);
   p->row_src = take(std::max<size_t>(M, 1) * 4);
   p->slot_row = take(std::max<long long>(A, 1) * 4);
+  p->sync = take((3 + E * 2) * 4);
   const size_t act = fp8 ? 1 : 2;
   // permuted x: bf16 copy (bf16 PREFILL) or e4m3 codes (both e4m3 paths);
   // bf16 DECODE reads the token rows of x in place
   // (e4m3 DECODE: one row per token, not per assignment)
-  const size_t xrows = (fp8 && p->path == MOE_PATH_DECODE) ? static_cast<size_t>(T) : M;
+  const size_t xrows = (fp8 && streaming) ? static_cast<size_t>(T) : M;
   p->xa = (p->path == MOE_PATH_PREFILL || fp8) ? take(xrows * H * act) : none;
   p->xs = fp8 ? take(xrows * (H / 128) * 4) : none;
   p->h = take(M * I * act);
   p->hs = fp8 ? take(M * (I / 128) * 4) : none;
-  p->hf = (fp8 && p->path == MOE_PATH_DECODE) ? take(M * I * 4) : none;
+  p->hf = (fp8 && streaming) ? take(M * I * 4) : none;
   p->y = take(M * H * 2);
   p->total = off;
   return true;
@@ -217,13 +221,18 @@ moe_status forward_impl(const moe_shape* shape, const void* x, const int32_t* to
   if (!validate_shape(shape)) return MOE_ERR_INVALID_ARG;
   if (!(n_events == 0 || (n_events == 5 && events != nullptr))) return MOE_ERR_INVALID_ARG;
   const bool fp8 = shape->wdtype == MOE_DT_E4M3;
-  if (fp8 && (sw_gate_up == nullptr || sw_down == nullptr)) return MOE_ERR_SCALE_FORMAT;
+  const bool fp4 = shape->wdtype == MOE_DT_E2M1;
+  if ((fp8 || fp4) && (sw_gate_up == nullptr || sw_down == nullptr)) return MOE_ERR_SCALE_FORMAT;
   Plan plan;
   if (!make_plan(shape, &plan)) return MOE_ERR_INVALID_ARG;
+  // e2m1 PREFILL: the down tile spans 256 columns of y
+  if (fp4 && plan.path == MOE_PATH_PREFILL && (!fp4_gemm_available() || shape->H % 256 != 0))
+    return MOE_ERR_UNSUPPORTED;
   // e4m3 PREFILL: the down tile spans two 128-column scale blocks
   if (fp8 && plan.path == MOE_PATH_PREFILL && (!e4m3_path_available() || shape->H % 256 != 0))
     return MOE_ERR_UNSUPPORTED;
   if (plan.path == MOE_PATH_DECODE && !decode_supported(shape)) return MOE_ERR_UNSUPPORTED;
+  if (plan.path == MOE_PATH_FUSED && !fused_supported(shape)) return MOE_ERR_UNSUPPORTED;
   if (shape->T == 0) return MOE_OK;
   if (x == nullptr || topk_idx == nullptr || topk_w == nullptr || w_gate_up == nullptr || w_down == nullptr ||
       out == nullptr || workspace == nullptr)
@@ -242,10 +251,21 @@ moe_status forward_impl(const moe_shape* shape, const void* x, const int32_t* to
   };
 
   if (!mark(0)) return MOE_ERR_CUDA;
+  if (plan.path == MOE_PATH_FUSED) {
+    // one launch: its time shows as the gate/up stage (events 1..2)
+    if (!mark(1)) return MOE_ERR_CUDA;
+    if (launch_fused_decode(shape, plan, x, topk_idx, topk_w, w_gate_up, w_down, out, ws, sms, st) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    return mark(2) && mark(3) && mark(4) ? MOE_OK : MOE_ERR_CUDA;
+  }
   if (launch_permute(shape, plan, topk_idx, x, ws, st) != cudaSuccess) return MOE_ERR_CUDA;
   if (!mark(1)) return MOE_ERR_CUDA;
   cudaError_t err;
-  if (plan.path == MOE_PATH_DECODE && fp8) {
+  if (plan.path == MOE_PATH_DECODE && fp4) {
+    err = launch_decode_fp4(shape, plan, x, w_gate_up, w_down, sw_gate_up, sw_down, ws, 0, sms, st);
+    if (err != cudaSuccess || !mark(2)) return MOE_ERR_CUDA;
+    err = launch_decode_fp4(shape, plan, x, w_gate_up, w_down, sw_gate_up, sw_down, ws, 1, sms, st);
+  } else if (plan.path == MOE_PATH_DECODE && fp8) {
     err = launch_decode_e4m3(shape, plan, w_gate_up, w_down, sw_gate_up, sw_down, ws, 0, sms, st);
     if (err != cudaSuccess || !mark(2)) return MOE_ERR_CUDA;
     err = launch_decode_e4m3(shape, plan, w_gate_up, w_down, sw_gate_up, sw_down, ws, 1, sms, st);
@@ -253,6 +273,10 @@ moe_status forward_impl(const moe_shape* shape, const void* x, const int32_t* to
     err = launch_decode(shape, plan, x, w_gate_up, w_down, ws, 0, sms, st);
     if (err != cudaSuccess || !mark(2)) return MOE_ERR_CUDA;
     err = launch_decode(shape, plan, x, w_gate_up, w_down, ws, 1, sms, st);
+  } else if (fp4) {
+    err = launch_gemm_fp4(shape, plan, w_gate_up, w_down, sw_gate_up, sw_down, ws, 0, sms, st);
+    if (err != cudaSuccess || !mark(2)) return MOE_ERR_CUDA;
+    err = launch_gemm_fp4(shape, plan, w_gate_up, w_down, sw_gate_up, sw_down, ws, 1, sms, st);
   } else if (!fp8) {
     // gate/up: single-CTA 128x256 tiles; down: CTA-pair 256x256 tiles when
     // H allows (each measured the faster of the two on the prefill-shaped and

@@ -15,6 +15,9 @@ constexpr int kTileM = 128;        // rows per expert tile on the PREFILL path
 constexpr int kPermuteTokens = 256;  // tokens per block in the permute kernels
 constexpr int kSmallPermuteT = 256;  // T up to this uses the single-block permute
 constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;  // bounded waits give up after 2 s
+constexpr size_t kSmemLimit = 232448;  // dynamic shared memory a B200 CTA may opt in to (227 KB)
+constexpr int kFusedMaxTokens = 256;         // FUSED path: one token per thread of a block
+constexpr int kFusedMaxAssignments = 2048;   // FUSED path: T*k held in every block's shared memory
 
 // Limit of every bounded device wait (kDefaultTimeoutNs unless a test set
 // another through moe_set_test_hooks), and that entry point's switch that makes
@@ -29,8 +32,15 @@ struct Plan {
   int64_t m_rows;  // row capacity of the permuted buffers
   int nblk;        // permute blocks of kPermuteTokens tokens
   size_t status, hdr, block_counts, cnt, mt_base, pt_base, touched, local_rank, row_src, slot_row;
+  size_t sync;  // FUSED path: task queues and per-expert completion counters (3 + 2E ints)
   size_t xa, xs, h, hs, hf, y, total;  // hf: fp32 h of the e4m3 DECODE path
 };
+
+// Words of the status block (workspace offset `status`), all zeroed by the
+// permute stage before the expert GEMMs run: the device status word, then one
+// dynamic tile counter per GEMM launch (gate/up, down).
+constexpr int kStatusTileCounter = 1;
+constexpr int kStatusWordsZeroed = 4;
 
 // Header words written on the device by the permute stage.
 enum HdrWord { kHdrMTiles = 0, kHdrTouched = 1, kHdrRows = 2, kHdrPairs = 3 };
@@ -74,9 +84,28 @@ cudaError_t launch_decode_e4m3(const moe_shape* s, const Plan& p, const void* w_
 cudaError_t launch_combine(const moe_shape* s, const Plan& p, const float* topk_w, void* out, uint8_t* ws,
                            cudaStream_t st);
 
+// FP4 (e2m1) experts on the DECODE path: which = 0 gate/up, 1 down.
+cudaError_t launch_decode_fp4(const moe_shape* s, const Plan& p, const void* x, const void* w_gate_up,
+                              const void* w_down, const uint8_t* sw_gate_up, const uint8_t* sw_down, uint8_t* ws,
+                              int which, int num_sms, cudaStream_t st);
+// FP4 experts on the PREFILL path (weights widened to bf16 in shared memory).
+bool fp4_gemm_available();
+cudaError_t launch_gemm_fp4(const moe_shape* s, const Plan& p, const void* w_gate_up, const void* w_down,
+                            const uint8_t* sw_gate_up, const uint8_t* sw_down, uint8_t* ws, int which, int num_sms,
+                            cudaStream_t st);
+
+// The FUSED path (bf16 experts): permute, gate/up, down and combine in one launch.
+bool fused_supported(const moe_shape* s);
+cudaError_t launch_fused_decode(const moe_shape* s, const Plan& p, const void* x, const int* topk_idx,
+                                const float* topk_w, const void* w_gate_up, const void* w_down, void* out,
+                                uint8_t* ws, int num_sms, cudaStream_t st);
+
 // Tensor-map encoding through the driver entry point (no link-time libcuda dependency).
+// 128-byte swizzle by default (every operand tile and bf16 output tile); the
+// 64-byte swizzle for tiles of 64-byte rows.
 bool encode_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, size_t elem_bytes, const void* base,
-                          uint64_t inner, uint64_t outer, uint32_t box_inner, uint32_t box_outer);
+                          uint64_t inner, uint64_t outer, uint32_t box_inner, uint32_t box_outer,
+                          CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B);
 
 int device_sm_count();
 

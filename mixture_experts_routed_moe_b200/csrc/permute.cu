@@ -428,7 +428,7 @@ cudaError_t launch_permute(const moe_shape* s, const Plan& p, const int* topk_id
     return cudaGetLastError();
   };
 
-  cudaError_t err = cudaMemsetAsync(status, 0, sizeof(int), st);
+  cudaError_t err = cudaMemsetAsync(status, 0, kStatusWordsZeroed * sizeof(int), st);
   if (err != cudaSuccess) return err;
   if (T <= kSmallPermuteT) {
     permute_small_kernel<<<1, 1024, mask_bytes, st>>>(topk_idx, T, k, E, p.bm, cnt, mt_base, pt_base, touched, hdr,
