@@ -47,14 +47,23 @@ typedef enum {
 } moe_status;
 
 /* Expert weight type. */
-typedef enum { MOE_DT_BF16 = 0, MOE_DT_E4M3 = 1 } moe_wdtype;
+typedef enum {
+  MOE_DT_BF16 = 0, /* bf16 weights */
+  MOE_DT_E4M3 = 1, /* e4m3 codes, one UE8M0 scale per 128x128 block; activations quantised 1x128 */
+  MOE_DT_E2M1 = 2  /* FP4: e2m1 codes two per byte (even element in the low nibble), one UE8M0
+                      scale per row and 32 consecutive elements along the reduction
+                      dimension; activations stay bf16 */
+} moe_wdtype;
 
 /* Which execution of the expert matmuls to use (the page's decode-stage switch:
  * small token counts run better on a per-token form than on grouped GEMM tiles). */
 typedef enum {
   MOE_PATH_AUTO = 0,    /* DECODE when T*k <= 4*E, else PREFILL */
   MOE_PATH_PREFILL = 1, /* expert-major permute + tcgen05 grouped GEMMs */
-  MOE_PATH_DECODE = 2   /* weight-streaming kernels, no tile padding */
+  MOE_PATH_DECODE = 2,  /* weight-streaming kernels, no tile padding */
+  MOE_PATH_FUSED = 3    /* the DECODE path's permute, gate/up, down and combine in one
+                           launch (section "Fused Mega MoE on Blackwell", on one GPU);
+                           bf16 experts, T <= 256 and T*k <= 2048, else MOE_ERR_UNSUPPORTED */
 } moe_path;
 
 /* Gate activation of the gated expert MLP (section "SonicMoE": SwiGLU, GeGLU
@@ -131,20 +140,30 @@ size_t moe_workspace_size(const moe_shape* shape);
  *   topk_idx   [T, k] int32, each row k distinct experts in [0, E)
  *   topk_w     [T, k] fp32
  *   w_gate_up  [E, 2I, H]: rows 0..I-1 of expert e are the gate projection,
- *              rows I..2I-1 the up projection. bf16, or e4m3 codes.
- *   w_down     [E, H, I], bf16 or e4m3 codes.
- *   sw_gate_up [E, 2I/128, H/128] UE8M0, one per 128x128 block (e4m3 only, else NULL)
- *   sw_down    [E, H/128, I/128] UE8M0 (e4m3 only, else NULL)
+ *              rows I..2I-1 the up projection. bf16, or e4m3 codes, or
+ *              e2m1 codes packed two per byte ([E, 2I, H/2] bytes).
+ *   w_down     [E, H, I], bf16 or e4m3 codes, or packed e2m1 ([E, H, I/2] bytes).
+ *   sw_gate_up e4m3: [E, 2I/128, H/128] UE8M0, one per 128x128 block;
+ *              e2m1: [E, 2I, H/32] UE8M0, one per row and 32 elements; bf16: NULL
+ *   sw_down    e4m3: [E, H/128, I/128]; e2m1: [E, H, I/32]; bf16: NULL
  *   out        [T, H] bf16 out
  *   workspace  >= moe_workspace_size(shape) bytes, 256-byte aligned; its
  *              previous contents do not matter. Calls that share a workspace
  *              must not overlap in time.
+ * On the FUSED path the permute, expert and combine stages share one launch;
+ * its layout, intermediates and results are those of the DECODE path.
  * Intermediates: h = act(gate) * up is rounded to bf16 and the expert output
  * y to bf16 (e4m3 experts: x and h are quantised per token and per 128-column
  * group with an fp32 scale amax/448, the FP8 reading of section "FP8 and FP4
  * quantized experts"; y stays bf16). The weighted sum runs in fp32 over j in
  * ascending order, so results are deterministic run to run.
- * Errors: MOE_ERR_SCALE_FORMAT when wdtype is e4m3 and a scale pointer is NULL
+ * e2m1 experts (section "FP8 and FP4 quantized experts": FP4-packed expert
+ * weights with UE8M0 scales) keep bf16 activations: every e2m1 value times a
+ * power of two is exact in bf16, so the layer is the bf16 layer on the
+ * dequantised weights. On the PREFILL path (weights widened to bf16 in shared
+ * memory ahead of the bf16 tensor-core MMA) H must be a multiple of 256, else
+ * MOE_ERR_UNSUPPORTED; the DECODE path takes any H that is a multiple of 128.
+ * Errors: MOE_ERR_SCALE_FORMAT when wdtype is e4m3 or e2m1 and a scale pointer is NULL
  * (the page's note: Blackwell kernels need UE8M0 scales and refuse plain float
  * ones instead of silently corrupting the output); MOE_ERR_UNSUPPORTED for
  * e4m3 weights on the PREFILL path with H not a multiple of 256 (the DECODE
@@ -202,8 +221,9 @@ moe_status moe_read_device_status(const void* workspace, void* stream);
  *    and returns. 0 restores the default of 2 s; otherwise 1 ms to 60 s.
  *  - stall_gate_up_loads: 1 makes the prefill gate/up GEMM's producer issue no
  *    loads, so the MMA issuer waits on a barrier nothing completes and gives up
- *    after wait_limit_ns; the rest of the call then runs on stale intermediates
- *    and its output is garbage. 0 turns it off.
+ *    after wait_limit_ns (on the FUSED path the gate/up tasks count no
+ *    completions, so the down tasks' waits give up); the rest of the call then
+ *    runs on stale intermediates and its output is garbage. 0 turns it off.
  *
  * Both are process-wide and read when a call is enqueued; do not change them
  * while other threads enqueue calls. Returns MOE_ERR_INVALID_ARG (and changes

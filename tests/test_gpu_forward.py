@@ -29,7 +29,7 @@ def _forward(wl, seed, path, idx=None, w=None, logits=None):
     return x, idx, w, W, out, ws
 
 
-@pytest.mark.parametrize("path", ["prefill", "decode"])
+@pytest.mark.parametrize("path", ["prefill", "decode", "fused"])
 @pytest.mark.parametrize("name", ["tiny", "decode"])
 def test_small_workloads_full_parity(name, path):
     wl = G.WORKLOADS[name]
@@ -55,9 +55,9 @@ def test_small_workloads_full_parity(name, path):
     assert_bf16_close(y, yref, "y")
 
 
-@pytest.mark.parametrize("path", ["prefill", "decode"])
-def test_paths_agree_and_are_deterministic(path):
-    wl = G.Workload("mid", 300, 256, 384, 16, 4)
+@pytest.mark.parametrize("path,T", [("prefill", 300), ("decode", 300), ("fused", 256)])
+def test_paths_agree_and_are_deterministic(path, T):
+    wl = G.Workload("mid", T, 256, 384, 16, 4)
     x, idx, w, W, out1, ws = _forward(wl, 11, path)
     out2, _ = moe.forward(x.cuda(), torch.from_numpy(idx).cuda(), torch.from_numpy(w).cuda(), W["w_gate_up"],
                           W["w_down"], path=path, workspace=ws)
@@ -80,9 +80,11 @@ EDGE_COUNTS = [
 ]
 
 
-@pytest.mark.parametrize("path", ["prefill", "decode"])
+@pytest.mark.parametrize("path", ["prefill", "decode", "fused"])
 @pytest.mark.parametrize("T,H,I,E,k,counts", EDGE_COUNTS)
 def test_edge_counts(T, H, I, E, k, counts, path):
+    if path == "fused" and T > 256:
+        pytest.skip("the fused path takes at most 256 tokens")
     wl = G.Workload("edge", T, H, I, E, k)
     idx, w = G.routed_inputs_with_counts(wl, counts, seed=T)
     x, idx_np, w_np, W, out, ws = _forward(wl, 3, path, idx=idx, w=w)
@@ -117,7 +119,7 @@ def test_bad_routing_index_is_reported_not_faulted():
     idx = idx.copy()
     idx[3, 1] = 4  # out of range
     idx[7, 1] = idx[7, 0]  # repeated expert
-    for path in ("prefill", "decode"):
+    for path in ("prefill", "decode", "fused"):
         out, ws = moe.forward(x.cuda(), torch.from_numpy(idx).cuda(), torch.from_numpy(w).cuda(), W["w_gate_up"],
                               W["w_down"], path=path)
         assert moe.read_device_status(ws) == -7
@@ -187,7 +189,7 @@ def test_full_size_bf16_every_token(name):
     assert_tokens_close(got, ref, TOKEN_REL_FRO, name)
 
 
-@pytest.mark.parametrize("path", ["prefill", "decode"])
+@pytest.mark.parametrize("path", ["prefill", "decode", "fused"])
 @pytest.mark.parametrize("name", ["tiny", "decode"])
 def test_combine_bit_exact_given_y(name, path):
     """The combine alone: fp32 fused multiply-adds in ascending j over the
@@ -197,13 +199,14 @@ def test_combine_bit_exact_given_y(name, path):
     check_combine_bit_exact(ws, moe.make_shape(wl.T, wl.H, wl.I, wl.E, wl.k, "bf16", path), w, out)
 
 
+@pytest.mark.parametrize("path", ["auto", "fused"])
 @pytest.mark.parametrize("name", ["tiny", "decode"])
-def test_graph_replay_matches_eager(name):
+def test_graph_replay_matches_eager(name, path):
     """MoEGraph (route + forward captured in a CUDA graph) gives the eager
     result on new inputs copied into its static buffers."""
     wl = G.WORKLOADS[name]
     W = G.make_weights(wl, 0, device="cuda")
-    layer = moe.MoELayer(W["w_gate_up"], W["w_down"], wl.k)
+    layer = moe.MoELayer(W["w_gate_up"], W["w_down"], wl.k, path=path)
     g = moe.MoEGraph(layer, wl.T)
     for seed in (21, 22):
         x, L = G.make_activations(wl, seed)
@@ -214,7 +217,7 @@ def test_graph_replay_matches_eager(name):
 
 
 @pytest.mark.parametrize("act", ["gelu", "relu"])
-@pytest.mark.parametrize("path", ["prefill", "decode"])
+@pytest.mark.parametrize("path", ["prefill", "decode", "fused"])
 @pytest.mark.parametrize("name", ["tiny", "decode"])
 def test_gated_activations(name, path, act):
     """GeGLU and ReGLU experts (section SonicMoE's silu/gelu/relu gates) on both paths."""
@@ -227,3 +230,44 @@ def test_gated_activations(name, path, act):
     assert moe.read_device_status(ws) == 0
     ref = O.moe_forward(x.float().numpy(), idx, w, ExpertView(W["w_gate_up"]), ExpertView(W["w_down"]), act=act)
     assert_bf16_close(out.float().cpu().numpy(), ref, f"{name}/{path}/{act}")
+
+
+def test_fused_path_equals_decode_path_bit_for_bit():
+    """The fused single-launch forward and the DECODE kernels compute the same
+    dot products in the same order: identical outputs, and an identical
+    permutation left in the workspace."""
+    wl = G.WORKLOADS["decode"]
+    x, idx, w, W, out_d, ws_d = _forward(wl, 41, "decode")
+    _, _, _, _, out_f, ws_f = _forward(wl, 41, "fused")
+    assert torch.equal(out_d, out_f)
+    shape = moe.make_shape(wl.T, wl.H, wl.I, wl.E, wl.k, "bf16", "fused")
+    assert moe.workspace_layout(shape).path == moe.PATH["fused"]
+    check_permutation(ws_f, shape, idx)
+
+
+def test_fused_path_bounded_wait_gives_up_cleanly():
+    """Gate/up tasks that never count as done (the test hook) leave every down
+    task's wait to run out: the call ends with MOE_ERR_DEVICE_TIMEOUT within
+    the short limit, not a hang, and the next call on the same context and
+    workspace gives the same bits as before."""
+    import time
+
+    wl = G.WORKLOADS["decode"]
+    x, L, W = device_inputs(wl, 43)
+    idx, w, _ = O.route(L.numpy(), wl.k)
+    args = (x.cuda(), torch.from_numpy(idx).cuda(), torch.from_numpy(w).cuda(), W["w_gate_up"], W["w_down"])
+    ref, ws = moe.forward(*args, path="fused")
+    torch.cuda.synchronize()
+    try:
+        moe.set_test_hooks(stall_gate_up_loads=True, wait_limit_ns=20_000_000)
+        t0 = time.perf_counter()
+        moe.forward(*args, path="fused", workspace=ws)
+        st = moe.read_device_status(ws)
+        elapsed = time.perf_counter() - t0
+    finally:
+        moe.set_test_hooks()
+    assert st == -6
+    assert elapsed < 1.0
+    again, _ = moe.forward(*args, path="fused", workspace=ws)
+    assert moe.read_device_status(ws) == 0
+    assert torch.equal(again, ref)
