@@ -23,8 +23,8 @@ STATUS = {
     -4: "MOE_ERR_WORKSPACE", -5: "MOE_ERR_CUDA", -6: "MOE_ERR_DEVICE_TIMEOUT", -7: "MOE_ERR_DEVICE_INDEX",
     -8: "MOE_ERR_SCRATCH_LIMIT",
 }
-WDTYPE = {"bf16": 0, "e4m3": 1}
-PATH = {"auto": 0, "prefill": 1, "decode": 2}
+WDTYPE = {"bf16": 0, "e4m3": 1, "e2m1": 2}
+PATH = {"auto": 0, "prefill": 1, "decode": 2, "fused": 3}
 ACT = {"silu": 0, "gelu": 1, "relu": 2}
 PATH_NAMES = {v: k for k, v in PATH.items()}
 EXPORTS = ["moe_route", "moe_workspace_size", "moe_forward", "moe_forward_timed", "moe_workspace_query",
@@ -193,21 +193,26 @@ def _check_forward_args(x, topk_idx, topk_w, w_gate_up, w_down, sw_gate_up, sw_d
     k = topk_idx.shape[1]
     _need(topk_idx, "topk_idx", (torch.int32,), 2, (T, k), cuda=False)
     _need(topk_w, "topk_w", (torch.float32,), 2, (T, k), cuda=False)
-    wtypes = (torch.bfloat16,) + ((_FLOAT8,) if _FLOAT8 is not None else ())
+    # bf16 weights, e4m3 codes (float8_e4m3fn) or packed e2m1 codes (uint8, two per byte)
+    wtypes = (torch.bfloat16, torch.uint8) + ((_FLOAT8,) if _FLOAT8 is not None else ())
     _need(w_gate_up, "w_gate_up", wtypes, 3, cuda=False)
     E, twoI = w_gate_up.shape[0], w_gate_up.shape[1]
     if twoI % 2 != 0:
         raise ValueError(f"w_gate_up: {twoI} rows per expert, expected 2*I (gate rows, then up rows)")
     I = twoI // 2
-    _need(w_gate_up, "w_gate_up", wtypes, 3, (E, 2 * I, H), cuda=False)
-    _need(w_down, "w_down", (w_gate_up.dtype,), 3, (E, H, I), cuda=False)
     fp8 = _FLOAT8 is not None and w_gate_up.dtype == _FLOAT8
-    if fp8:
-        # UE8M0 bytes, one per 128x128 weight block (None: the library refuses with MOE_ERR_SCALE_FORMAT)
+    fp4 = w_gate_up.dtype == torch.uint8
+    pk = 2 if fp4 else 1  # elements per stored byte or element along the reduction dimension
+    _need(w_gate_up, "w_gate_up", wtypes, 3, (E, 2 * I, H // pk), cuda=False)
+    _need(w_down, "w_down", (w_gate_up.dtype,), 3, (E, H, I // pk), cuda=False)
+    if fp8 or fp4:
+        # UE8M0 bytes: one per 128x128 block (e4m3) or per row and 32 elements (e2m1);
+        # None makes the library refuse with MOE_ERR_SCALE_FORMAT
+        g_gu, g_d = ((2 * I // 128, H // 128), (H // 128, I // 128)) if fp8 else ((2 * I, H // 32), (H, I // 32))
         if sw_gate_up is not None:
-            _need(sw_gate_up, "sw_gate_up", (torch.uint8,), 3, (E, 2 * I // 128, H // 128), cuda=False)
+            _need(sw_gate_up, "sw_gate_up", (torch.uint8,), 3, (E,) + g_gu, cuda=False)
         if sw_down is not None:
-            _need(sw_down, "sw_down", (torch.uint8,), 3, (E, H // 128, I // 128), cuda=False)
+            _need(sw_down, "sw_down", (torch.uint8,), 3, (E,) + g_d, cuda=False)
     elif sw_gate_up is not None or sw_down is not None:
         raise ValueError("block scales were given for bf16 experts")
     if out is not None:
@@ -216,7 +221,7 @@ def _check_forward_args(x, topk_idx, topk_w, w_gate_up, w_down, sw_gate_up, sw_d
         _need(workspace, "workspace", (torch.uint8,), 1, cuda=False)
     _same_device(x.device, topk_idx=topk_idx, topk_w=topk_w, w_gate_up=w_gate_up, w_down=w_down,
                  sw_gate_up=sw_gate_up, sw_down=sw_down, out=out, workspace=workspace)
-    return T, H, I, E, k, ("e4m3" if fp8 else "bf16")
+    return T, H, I, E, k, ("e4m3" if fp8 else "e2m1" if fp4 else "bf16")
 
 
 def forward(x, topk_idx, topk_w, w_gate_up, w_down, sw_gate_up=None, sw_down=None, out=None, workspace=None,
@@ -316,12 +321,13 @@ class MoELayer:
         self.w_gate_up, self.w_down = w_gate_up, w_down
         self.sw_gate_up, self.sw_down = sw_gate_up, sw_down
         self.k, self.path, self.act = int(k), path, act
-        self.E, twoI, self.H = w_gate_up.shape
+        self.E, twoI = w_gate_up.shape[0], w_gate_up.shape[1]
+        self.H = w_down.shape[1]
         self.I = twoI // 2
         self._ws = {}
 
     def _workspace(self, T, device):
-        wdtype = "e4m3" if self.w_gate_up.dtype == torch.float8_e4m3fn else "bf16"
+        wdtype = {torch.float8_e4m3fn: "e4m3", torch.uint8: "e2m1"}.get(self.w_gate_up.dtype, "bf16")
         shape = make_shape(T, self.H, self.I, self.E, self.k, wdtype, self.path, self.act)
         key = (T, str(device))
         if key not in self._ws:

@@ -17,6 +17,13 @@ Distributions: hidden states N(0,1) rounded to bf16; expert weights
 N(0, 0.02) rounded to bf16 (or quantised to e4m3, see below); router logits
 N(0,1) in fp32.
 
+FP4 weights (e2m1, the FP4-packed experts of the same section) are prepared
+the same way per row and block of 32 consecutive columns: the smallest s
+with 6 * 2^s >= amax, UE8M0 byte s + 127, codes = w / 2^s rounded to the
+nearest e2m1 value (ties to the even code), two codes per byte with the even
+column in the low nibble. torch has no e2m1 cast, so the rounding is done
+here with plain tensor arithmetic on the e2m1 grid.
+
 Hidden states and logits come from numpy's PCG64 seeded with ``seed`` and do
 not depend on the device. Expert weights are drawn per expert from a torch
 generator on the device that will hold them (seed ``seed * 100003 + e``), so a
@@ -41,6 +48,9 @@ import torch
 WEIGHT_STD = 0.02
 E4M3_MAX = 448.0
 QBLOCK = 128  # weight scale block (rows and columns)
+E2M1_MAX = 6.0
+FP4_BLOCK = 32  # FP4 weight scale block (columns of one row)
+_E2M1_GRID = (0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0)
 
 
 @dataclasses.dataclass(frozen=True)
@@ -51,7 +61,7 @@ class Workload:
     I: int
     E: int
     k: int
-    wdtype: str = "bf16"  # "bf16" or "e4m3"
+    wdtype: str = "bf16"  # "bf16", "e4m3" or "e2m1"
     router_bias: bool = False
 
     @property
@@ -75,9 +85,12 @@ WORKLOADS = {
     "skewed": Workload("skewed", 4096, 4096, 14336, 8, 2, router_bias=True),
     # the FP8 layer's experts at decode size: 16 tokens, weight-streaming path
     "fp8_decode": Workload("fp8_decode", 16, 7168, 2048, 256, 8, wdtype="e4m3"),
+    # the large layer's shape with FP4 (e2m1) experts, at prefill and decode size
+    "fp4": Workload("fp4", 4096, 7168, 2048, 256, 8, wdtype="e2m1"),
+    "fp4_decode": Workload("fp4_decode", 16, 7168, 2048, 256, 8, wdtype="e2m1"),
 }
 # the seed of each named workload is its position in this list
-WORKLOAD_ORDER = ["tiny", "decode", "prefill", "fp8", "skewed", "fp8_decode"]
+WORKLOAD_ORDER = ["tiny", "decode", "prefill", "fp8", "skewed", "fp8_decode", "fp4", "fp4_decode"]
 
 
 def default_seed(wl: Workload) -> int:
@@ -125,6 +138,26 @@ def quantize_weight_blocks(w: torch.Tensor):
     return q, (s + 127).to(torch.uint8)
 
 
+def quantize_fp4_rows(w: torch.Tensor):
+    """Checkpoint-style FP4 quantisation of one [R, C] fp32 matrix (C a
+    multiple of 32). Returns (packed uint8 [R, C/2], ue8m0 uint8 [R, C/32])."""
+    R, C = w.shape
+    blk = w.reshape(R, C // FP4_BLOCK, FP4_BLOCK)
+    amax = blk.abs().amax(dim=2)
+    ratio = amax / E2M1_MAX
+    m, ex = torch.frexp(ratio)
+    s = ex - (m == 0.5).to(ex.dtype)  # smallest s with 2^s >= amax / 6
+    s = torch.where(amax > 0, s, torch.zeros_like(s))
+    q = blk / torch.ldexp(torch.ones_like(ratio), s)[:, :, None]
+    mag = q.abs().clamp(max=E2M1_MAX)
+    step = torch.where(mag < 2.0, 0.5, torch.where(mag < 4.0, 1.0, 2.0))
+    r = torch.minimum(torch.round(mag / step) * step, torch.full_like(mag, E2M1_MAX))  # round: ties to even
+    grid = torch.tensor(_E2M1_GRID, device=w.device)
+    code = torch.searchsorted(grid, r.contiguous()).to(torch.uint8) | (torch.signbit(q).to(torch.uint8) << 3)
+    code = code.reshape(R, C)
+    return (code[:, 0::2] | (code[:, 1::2] << 4)).contiguous(), (s + 127).to(torch.uint8)
+
+
 def make_weights(wl: Workload, seed: int, device="cpu"):
     """Expert weights on ``device``.
 
@@ -151,6 +184,16 @@ def make_weights(wl: Workload, seed: int, device="cpu"):
             wgu[e], sgu[e] = quantize_weight_blocks(_draw((2 * I, H), g, device))
             wd[e], sd[e] = quantize_weight_blocks(_draw((H, I), g, device))
         return dict(w_gate_up=wgu, w_down=wd, sw_gate_up=sgu, sw_down=sd)
+    if wl.wdtype == "e2m1":
+        wgu = torch.empty((E, 2 * I, H // 2), dtype=torch.uint8, device=device)
+        wd = torch.empty((E, H, I // 2), dtype=torch.uint8, device=device)
+        sgu = torch.empty((E, 2 * I, H // FP4_BLOCK), dtype=torch.uint8, device=device)
+        sd = torch.empty((E, H, I // FP4_BLOCK), dtype=torch.uint8, device=device)
+        for e in range(E):
+            g = _expert_generator(seed, e, device)
+            wgu[e], sgu[e] = quantize_fp4_rows(_draw((2 * I, H), g, device))
+            wd[e], sd[e] = quantize_fp4_rows(_draw((H, I), g, device))
+        return dict(w_gate_up=wgu, w_down=wd, sw_gate_up=sgu, sw_down=sd)
     raise ValueError(f"unknown weight dtype {wl.wdtype!r}")
 
 
@@ -161,6 +204,10 @@ def make_expert_weights(wl: Workload, seed: int, e: int, device="cpu"):
     b = _draw((wl.H, wl.I), g, device)
     if wl.wdtype == "bf16":
         return dict(w_gate_up=a.to(torch.bfloat16), w_down=b.to(torch.bfloat16))
+    if wl.wdtype == "e2m1":
+        qa, sa = quantize_fp4_rows(a)
+        qb, sb = quantize_fp4_rows(b)
+        return dict(w_gate_up=qa, w_down=qb, sw_gate_up=sa, sw_down=sb)
     qa, sa = quantize_weight_blocks(a)
     qb, sb = quantize_weight_blocks(b)
     return dict(w_gate_up=qa, w_down=qb, sw_gate_up=sa, sw_down=sb)
@@ -206,10 +253,12 @@ def flops_and_bytes(wl: Workload, touched_experts: int | None = None):
     """Algorithmic FLOPs and minimum HBM bytes of one forward (route excluded):
     touched expert weights + x read + out written."""
     E_t = wl.E if touched_experts is None else touched_experts
-    welem = 1 if wl.wdtype == "e4m3" else 2
-    wbytes = E_t * 3 * wl.H * wl.I * welem
+    welem = {"e4m3": 1.0, "e2m1": 0.5}.get(wl.wdtype, 2.0)
+    wbytes = int(E_t * 3 * wl.H * wl.I * welem)
     if wl.wdtype == "e4m3":
         wbytes += E_t * (2 * wl.I // QBLOCK * wl.H // QBLOCK + wl.H // QBLOCK * wl.I // QBLOCK)
+    if wl.wdtype == "e2m1":
+        wbytes += E_t * 3 * wl.H * wl.I // FP4_BLOCK
     act = wl.T * wl.H * 2 * 2
     return wl.flops(), wbytes + act
 
@@ -220,7 +269,8 @@ def ceil_div(a: int, b: int) -> int:
 
 __all__ = [
     "Workload", "WORKLOADS", "WORKLOAD_ORDER", "default_seed", "make_activations", "make_weights",
-    "make_expert_weights", "make_router_weights", "quantize_weight_blocks", "routed_inputs_with_counts",
+    "make_expert_weights", "make_router_weights", "quantize_weight_blocks", "quantize_fp4_rows",
+    "routed_inputs_with_counts",
     "flops_and_bytes",
     "router_bias", "ceil_div",
 ]

@@ -39,6 +39,15 @@ design notes):
   R5 aggregation: out[t] = sum_j w[t,j] * y[t,j] with the given fp32 weights.
   R6 permutation: expert-major, tokens ascending within an expert, each expert's
      block padded up to a multiple of BM rows (pad rows carry source -1).
+  R8 FP4 experts (section "FP8 and FP4 quantized experts": FP4-packed expert
+     weights with UE8M0 scales on Blackwell): weights are OCP MX e2m1 codes
+     (sign, 2 exponent bits with bias 1, 1 mantissa bit: magnitudes 0, 0.5,
+     1, 1.5, 2, 3, 4, 6), two per byte with the even element in the low
+     nibble, times 2^(byte-127) for each block of 32 consecutive elements
+     along the reduction dimension (the OCP MX block). The page names no
+     activation format for FP4 experts, so activations stay bf16 (weight-only
+     quantisation); every e2m1 value times a power of two is exact in bf16,
+     so the layer is the bf16 layer (R4) on the dequantised weights.
   R7 FP8 (section "FP8 and FP4 quantized experts", and its note on Blackwell
      UE8M0 scales): weights are e4m3 codes times 2^(byte-127) per 128x128
      block; activations are quantised per token, per 128-column group, with an
@@ -419,3 +428,90 @@ def moe_forward_fp8(x, topk_idx, topk_w, wgu_codes, wgu_sb, wd_codes, wd_sb,
 
     Y = _expert_loop(x, topk_idx, E, tokens, mlp)
     return combine(Y, np.asarray(topk_w)[tokens], "bf16")
+
+
+# ---------------------------------------------------------------------------
+# FP4 experts (reading R8)
+# ---------------------------------------------------------------------------
+
+E2M1_MAX = 6.0
+FP4_BLOCK = 32  # elements per UE8M0 scale, along the reduction dimension
+
+
+def _e2m1_value(c) -> np.ndarray:
+    """Float64 value of each 4-bit e2m1 code: sign bit 3, exponent field e
+    (bits 2..1, bias 1), mantissa m (bit 0); e = 0 is subnormal m * 0.5,
+    otherwise (1 + m/2) * 2^(e-1)."""
+    c = np.asarray(c, dtype=np.int64) & 0xF
+    s = np.where(c & 0x8, -1.0, 1.0)
+    e = (c >> 1) & 0x3
+    m = c & 0x1
+    return s * np.where(e == 0, m * 0.5, (1.0 + m / 2.0) * np.ldexp(1.0, e - 1))
+
+
+_E2M1_VALUES = _e2m1_value(np.arange(16))
+
+
+def e2m1_decode(codes) -> np.ndarray:
+    """Float64 values of 4-bit e2m1 codes (the table of all 16)."""
+    return _E2M1_VALUES[np.asarray(codes, dtype=np.uint8) & 0xF]
+
+
+def e2m1_round(v) -> np.ndarray:
+    """Nearest e2m1 value, ties to the even code (mantissa bit 0), magnitudes
+    above 6 saturating to 6; returns float64. The spacing is 0.5 below 2, 1 on
+    [2, 4) and 2 on [4, 6]."""
+    v = np.asarray(v, dtype=np.float64)
+    mag = np.minimum(np.abs(v), E2M1_MAX)
+    step = np.where(mag < 2.0, 0.5, np.where(mag < 4.0, 1.0, 2.0))
+    r = np.rint(mag / step) * step  # rint: ties to even multiples of the step
+    return np.copysign(np.minimum(r, E2M1_MAX), v)
+
+
+def e2m1_encode(v) -> np.ndarray:
+    """4-bit e2m1 codes (uint8 0..15) of float values v after :func:`e2m1_round`."""
+    r = e2m1_round(v)
+    mag = np.abs(r)
+    idx = np.searchsorted(_E2M1_VALUES[:8], mag)  # the 8 magnitudes are increasing
+    return (idx.astype(np.uint8) | (np.signbit(r).astype(np.uint8) << 3)).astype(np.uint8)
+
+
+def unpack_e2m1(packed) -> np.ndarray:
+    """4-bit codes [..., 2n] from bytes [..., n]: element 2i in the low nibble of byte i."""
+    b = np.asarray(packed, dtype=np.uint8)
+    out = np.empty(b.shape[:-1] + (2 * b.shape[-1],), dtype=np.uint8)
+    out[..., 0::2] = b & 0xF
+    out[..., 1::2] = b >> 4
+    return out
+
+
+def pack_e2m1(codes) -> np.ndarray:
+    """Bytes [..., n] from 4-bit codes [..., 2n] (inverse of :func:`unpack_e2m1`)."""
+    c = np.asarray(codes, dtype=np.uint8) & 0xF
+    return (c[..., 0::2] | (c[..., 1::2] << 4)).astype(np.uint8)
+
+
+def dequantize_fp4(packed, scale_bytes):
+    """Weights [R, C] of one FP4 expert matrix from packed e2m1 bytes [R, C/2]
+    and one UE8M0 byte per row and block of 32 columns [R, C/32]."""
+    q = e2m1_decode(unpack_e2m1(packed))
+    s = ue8m0_scale(scale_bytes)
+    R, C = q.shape
+    return (q.reshape(R, C // FP4_BLOCK, FP4_BLOCK) * s[:, :, None]).reshape(R, C)
+
+
+def moe_forward_fp4(x, topk_idx, topk_w, wgu_packed, wgu_sb, wd_packed, wd_sb, tokens=None, act: str = "silu"):
+    """Routed MoE forward for FP4 experts (reading R8): the bf16 forward on the
+    dequantised weights. Shapes: wgu_packed uint8 [E,2I,H/2], wgu_sb uint8
+    [E,2I,H/32], wd_packed uint8 [E,H,I/2], wd_sb uint8 [E,H,I/32]."""
+    E = len(wgu_packed) if not hasattr(wgu_packed, "shape") else wgu_packed.shape[0]
+
+    class _Deq:
+        def __init__(self, packed, sb):
+            self.packed, self.sb = packed, sb
+            self.shape = (E,)
+
+        def __getitem__(self, e):
+            return dequantize_fp4(self.packed[e], self.sb[e])
+
+    return moe_forward(x, topk_idx, topk_w, _Deq(wgu_packed, wgu_sb), _Deq(wd_packed, wd_sb), tokens=tokens, act=act)
