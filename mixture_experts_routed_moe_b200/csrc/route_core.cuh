@@ -4,75 +4,69 @@
 // in global memory) and the fused router GEMM (logits in shared memory), so
 // both give the same bits for the same logits.
 //
-// Each lane holds up to kPerLane logits (expert lane + 32*i). The warp
-// computes the fp32 softmax denominator over all E experts, then selects k
-// times the largest remaining logit (equal logits: lower index first) with a
-// shuffle reduction over (value, index), and finally renormalises the chosen
-// probabilities over the k. Selection compares the logits themselves, which
-// orders experts exactly as the softmax does.
+// Each lane holds up to kPerLane logits (expert lane + 32*i). The warp selects
+// k times the largest remaining logit (equal logits: lower index first):
+// every lane offers its best untaken (logit, expert), one warp max-reduction
+// over order-preserving integer keys of the logits finds the value and one
+// min-reduction over the experts offering it breaks ties. Selection compares
+// the logits themselves, which orders experts exactly as the softmax does.
+// The weights are the softmax probabilities renormalised over the k chosen
+// experts: w_j = exp(l_j - l_max) / sum_j' exp(l_j' - l_max), where the first
+// selected logit is l_max and the softmax denominator over all E experts
+// cancels. The sum is compensated (Kahan).
 #pragma once
 
 #include "moe_common.cuh"
 
 namespace moe {
 
-__device__ __forceinline__ bool route_beats(float v, int i, float bv, int bi) {
-  return v > bv || (v == bv && i < bi);
+// Order-preserving map of a (non-NaN) float to an unsigned key: larger floats
+// give larger keys, -0 and +0 the same one, and the inverse map is exact.
+__device__ __forceinline__ uint32_t route_key(float f) {
+  const uint32_t b = __float_as_uint(f == 0.0f ? 0.0f : f);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float route_key_value(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
 }
 
 // row: the token's E logits (global or shared memory); idx_out / w_out: its k slots.
 template <int kPerLane>
 __device__ __forceinline__ void route_token(const float* row, int E, int k, int lane, int* idx_out, float* w_out) {
   float v[kPerLane];
-  float vmax = -INFINITY;
 #pragma unroll
   for (int i = 0; i < kPerLane; ++i) {
     const int e = lane + 32 * i;
     v[i] = (e < E) ? row[e] : -INFINITY;
-    vmax = fmaxf(vmax, v[i]);
   }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
-
-  // softmax denominator over all experts (fp32)
-  float z = 0.f;
-#pragma unroll
-  for (int i = 0; i < kPerLane; ++i)
-    if (lane + 32 * i < E) z += expf(v[i] - vmax);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-
   uint32_t taken = 0;  // bit i: expert lane + 32*i already selected
-  float psum = 0.f, pcomp = 0.f;  // compensated (Kahan) sum of the chosen probabilities
+  float vmax = 0.f, psum = 0.f, pcomp = 0.f;
   for (int j = 0; j < k; ++j) {
-    float bv = -INFINITY;
+    // this lane's best untaken expert (i ascending keeps the lower index on ties)
+    uint32_t key = 0;  // below every logit's key: no candidate
     int bi = 0x7fffffff;
 #pragma unroll
     for (int i = 0; i < kPerLane; ++i) {
       const int e = lane + 32 * i;
-      if (e < E && !(taken & (1u << i)) && route_beats(v[i], e, bv, bi)) {
-        bv = v[i];
+      const uint32_t ki = route_key(v[i]);
+      if (e < E && !(taken & (1u << i)) && (ki > key || bi == 0x7fffffff)) {
+        key = ki;
         bi = e;
       }
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (route_beats(ov, oi, bv, bi)) {
-        bv = ov;
-        bi = oi;
-      }
-    }
-    // the owner lane marks the winner as taken
-    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-    const float p = expf(bv - vmax) / z;  // softmax probability of the winner
+    const uint32_t kmax = __reduce_max_sync(0xffffffffu, key);
+    const int win = static_cast<int>(
+        __reduce_min_sync(0xffffffffu, key == kmax ? static_cast<uint32_t>(bi) : 0x7fffffffu));
+    if ((win & 31) == lane) taken |= 1u << (win >> 5);
+    const float bv = route_key_value(kmax);
+    if (j == 0) vmax = bv;
+    const float p = expf(bv - vmax);  // exp(l_j - l_max): the softmax numerator
     const float yk = p - pcomp;
     const float tk = psum + yk;
     pcomp = (tk - psum) - yk;
     psum = tk;
     if (lane == 0) {
-      idx_out[j] = bi;
+      idx_out[j] = win;
       w_out[j] = p;
     }
   }

@@ -16,8 +16,11 @@
 // token. Rows beyond E in the padded tile are zero (TMA fills out-of-range rows
 // with zeros) and are never read by the routing.
 //
-// Warp roles (192 threads): warp 0 TMA producer, warp 1 TMEM allocator and
-// MMA issuer, warps 2..5 epilogue (warp w reads TMEM lanes 32*(w%4)..+31).
+// Warp roles (512 threads): warp 0 TMA producer, warp 1 TMEM allocator and
+// MMA issuer, warps 2..5 epilogue (warp w reads TMEM lanes 32*(w%4)..+31);
+// then all sixteen warps route the tile's 128 tokens, eight each (the routing
+// of a token is a chain of warp reductions, so more warps in flight is what
+// shortens the tile's tail).
 #include "moe_common.cuh"
 #include "moe_internal.h"
 #include "route_core.cuh"
@@ -28,7 +31,7 @@ namespace {
 constexpr int kBK = 64;       // K elements per stage (128 bytes of bf16: one swizzle row)
 constexpr int kMaxStages = 8;
 constexpr size_t kRingBytes = 192 * 1024;  // shared memory for the TMA ring
-constexpr int kThreads = 192;
+constexpr int kThreads = 512;
 constexpr int kRows = 128;    // tokens per CTA (MMA M)
 constexpr int kA = kRows * kBK * 2;  // 16 KB
 
@@ -183,7 +186,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
 
-  // ---------------- routing: one warp per token of the tile ----------------
+  // ---------------- routing: one warp per token of the tile, every warp ----------------
   const int rows = min(kRows, p.T - row0);
   if (*s_abort != 0) {
     // a bounded wait gave up (never in normal operation): mark the tokens
