@@ -54,7 +54,7 @@ from mixture_experts_routed_moe_b200 import inputs as G  # noqa: E402
 METRIC = "MoE layer tokens/sec and TFLOP/s (% of BF16/FP8 peak or HBM BW) on 1 B200"
 DEFAULT_WORKLOAD = "fp8"
 # measured after the headline, in this order, under "per_config"
-OTHER_WORKLOADS = ["tiny", "decode", "prefill", "skewed", "fp8_decode"]
+OTHER_WORKLOADS = ["tiny", "decode", "prefill", "skewed", "fp8_decode", "fp4", "fp4_decode"]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FLUSH_BYTES = 256 << 20
 
@@ -190,9 +190,7 @@ class _HostExperts:
 
     def __init__(self, wl, seed, experts, name, codes=False):
         dev = "cuda" if torch.cuda.is_available() else "cpu"
-        self.shape = {"w_gate_up": (wl.E, 2 * wl.I, wl.H), "w_down": (wl.E, wl.H, wl.I),
-                      "sw_gate_up": (wl.E, 2 * wl.I // 128, wl.H // 128),
-                      "sw_down": (wl.E, wl.H // 128, wl.I // 128)}[name]
+        self.shape = (wl.E,)
         self.d = {}
         for e in experts:
             t = G.make_expert_weights(wl, seed, int(e), device=dev)[name].cpu()
@@ -215,8 +213,9 @@ def oracle_sample_rate(wl, seed, n_tokens, steps=1, warmup=0, min_seconds=0.0):
     idx0, _, _ = O.route(L, wl.k)
     experts = np.unique(idx0)
     fp8 = wl.wdtype == "e4m3"
-    V = {n: _HostExperts(wl, seed, experts, n, codes=fp8) for n in
-         (("w_gate_up", "w_down", "sw_gate_up", "sw_down") if fp8 else ("w_gate_up", "w_down"))}
+    fp4 = wl.wdtype == "e2m1"
+    V = {n: _HostExperts(wl, seed, experts, n, codes=fp8 or fp4) for n in
+         (("w_gate_up", "w_down", "sw_gate_up", "sw_down") if fp8 or fp4 else ("w_gate_up", "w_down"))}
     times = []
     i = 0
     while i < warmup + steps or (sum(times) < min_seconds and len(times) < 200):
@@ -224,6 +223,8 @@ def oracle_sample_rate(wl, seed, n_tokens, steps=1, warmup=0, min_seconds=0.0):
         idx, w, _ = O.route(L, wl.k)
         if fp8:
             O.moe_forward_fp8(xs, idx, w, V["w_gate_up"], V["sw_gate_up"], V["w_down"], V["sw_down"])
+        elif fp4:
+            O.moe_forward_fp4(xs, idx, w, V["w_gate_up"], V["sw_gate_up"], V["w_down"], V["sw_down"])
         else:
             O.moe_forward(xs, idx, w, V["w_gate_up"], V["w_down"])
         if i >= warmup:
@@ -243,7 +244,7 @@ def oracle_sample_tokens(wl):
     """Tokens per oracle sample, sized for roughly 10-30 s of CPU work: the
     eager loop's cost is dominated by converting each touched expert's weights
     to float64 (dequantising them for e4m3), about 3*H*I elements per expert."""
-    per_expert = 3 * wl.H * wl.I * (4 if wl.wdtype == "e4m3" else 1)
+    per_expert = 3 * wl.H * wl.I * (4 if wl.wdtype in ("e4m3", "e2m1") else 1)
     budget = 3.0e9  # element conversions
     experts = max(1, int(budget // per_expert))
     return max(1, min(wl.T, 16, experts // wl.k))
@@ -281,24 +282,40 @@ def workload_config(wl, path):
 def stage_roofline(wl, path, stage_ms, n_touched, peaks, peak_src):
     """Roofline of the slowest stage (its one kernel), algorithmic work per launch."""
     A, H, I = wl.A, wl.H, wl.I
-    welem = 1 if wl.wdtype == "e4m3" else 2
+    welem = {"e4m3": 1, "e2m1": 0.5}.get(wl.wdtype, 2)
+    fp4 = wl.wdtype == "e2m1"
     names = {1: "gate_up", 2: "down"}
     s = max((1, 2), key=lambda i: stage_ms[i])
     dur_s = stage_ms[s] / 1e3
-    if path == "decode":
+    if path == "fused":
+        # one launch does the whole forward (its time is the gate_up stage):
+        # every touched expert's weights, x read and out written once
+        dur_s = stage_ms[1] / 1e3
+        byts = n_touched * 3 * I * H * 2 + wl.T * H * 2 * 2
+        ach = byts / dur_s / 1e9
+        peak = peaks["hbm_gbs"]
+        out = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
+               "kernel": "fused_decode_kernel", "stage": "fused", "algorithmic_bytes": byts}
+        kern, src = "fused_decode_kernel", "fused_decode.cu"
+    elif path == "decode":
         fp8 = wl.wdtype == "e4m3"
-        # e4m3: one UE8M0 byte per 128x128 weight block, h stored as e4m3 codes
-        s_gu = n_touched * (2 * I // 128) * (H // 128) if fp8 else 0
-        s_d = n_touched * (H // 128) * (I // 128) if fp8 else 0
-        h_bytes = A * I * welem
+        # e4m3: one UE8M0 byte per 128x128 weight block, h stored as e4m3 codes;
+        # e2m1: one UE8M0 byte per 32 weights, h stored as bf16
+        s_gu = (n_touched * (2 * I // 128) * (H // 128) if fp8 else
+                n_touched * 2 * I * (H // 32) if fp4 else 0)
+        s_d = (n_touched * (H // 128) * (I // 128) if fp8 else
+               n_touched * H * (I // 32) if fp4 else 0)
+        h_bytes = A * I * (1 if fp8 else 2)
         if s == 1:
-            byts = n_touched * 2 * I * H * welem + s_gu + wl.T * H * 2 + h_bytes
-            kern, src = (("decode_e4m3_gate_up_kernel", "decode_e4m3.cu") if fp8
-                         else ("decode_gate_up_kernel", "decode.cu"))
+            byts = int(n_touched * 2 * I * H * welem) + s_gu + wl.T * H * 2 + h_bytes
+            kern, src = (("decode_e4m3_gate_up_kernel", "decode_e4m3.cu") if fp8 else
+                         ("decode_fp4_gate_up_kernel", "decode_fp4.cu") if fp4 else
+                         ("decode_gate_up_kernel", "decode.cu"))
         else:
-            byts = n_touched * H * I * welem + s_d + h_bytes + A * H * 2
-            kern, src = (("decode_e4m3_down_kernel", "decode_e4m3.cu") if fp8
-                         else ("decode_down_kernel", "decode.cu"))
+            byts = int(n_touched * H * I * welem) + s_d + h_bytes + A * H * 2
+            kern, src = (("decode_e4m3_down_kernel", "decode_e4m3.cu") if fp8 else
+                         ("decode_fp4_down_kernel", "decode_fp4.cu") if fp4 else
+                         ("decode_down_kernel", "decode.cu"))
         ach = byts / dur_s / 1e9
         peak = peaks["hbm_gbs"]
         out = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
@@ -310,13 +327,21 @@ def stage_roofline(wl, path, stage_ms, n_touched, peaks, peak_src):
         # and is HBM-bound
         flops = (4 if s == 1 else 2) * A * H * I
         fp8 = wl.wdtype == "e4m3"
+        aelem = 1 if fp8 else 2  # activation bytes (e4m3 codes, or bf16 for the bf16 and e2m1 layers)
         if s == 1:
-            byts = (n_touched * 2 * I * H * welem + A * H * welem + A * I * welem
-                    + (n_touched * (2 * I // 128) * (H // 128) + A * (H // 128) * 4 + A * (I // 128) * 4 if fp8 else 0))
+            byts = int(n_touched * 2 * I * H * welem + A * H * aelem + A * I * aelem
+                       + (n_touched * (2 * I // 128) * (H // 128) + A * (H // 128) * 4 + A * (I // 128) * 4 if fp8
+                          else n_touched * 2 * I * (H // 32) if fp4 else 0))
         else:
-            byts = (n_touched * H * I * welem + A * I * welem + A * H * 2
-                    + (n_touched * (H // 128) * (I // 128) + A * (I // 128) * 4 if fp8 else 0))
-        if fp8:
+            byts = int(n_touched * H * I * welem + A * I * aelem + A * H * 2
+                       + (n_touched * (H // 128) * (I // 128) + A * (I // 128) * 4 if fp8
+                          else n_touched * H * (I // 32) if fp4 else 0))
+        if fp4:
+            # the codes are widened to bf16 ahead of bf16 MMAs
+            tpeak, how = peaks["bf16_tflops"], "measured bf16 burst (the MMA is bf16)"
+            kern, src = ("grouped_gemm_fp4_kernel<1,0>" if s == 1 else "grouped_gemm_fp4_kernel<0,0>"), \
+                "gemm_fp4.cu"
+        elif fp8:
             tpeak, how = 2.0 * peaks["bf16_tflops"], "2x measured bf16 (nominal fp8:bf16 ratio)"
             kern, src = ("grouped_gemm_e4m3_kernel<true>" if s == 1 else "grouped_gemm_e4m3_kernel<false>"), \
                 "gemm_e4m3.cu"
@@ -404,10 +429,10 @@ def measure(moe, wl, args, world, rank, local, peaks, peak_src):
     x, logits = G.make_activations(wl, seed)
     W = G.make_weights(wl, seed, device=dev)
     xd, ld = x.to(dev), logits.to(dev)
-    layer = moe.MoELayer(W["w_gate_up"], W["w_down"], wl.k, W.get("sw_gate_up"), W.get("sw_down"))
+    layer = moe.MoELayer(W["w_gate_up"], W["w_down"], wl.k, W.get("sw_gate_up"), W.get("sw_down"), path=args.path)
     out = torch.empty((wl.T, wl.H), dtype=torch.bfloat16, device=dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    shape = moe.make_shape(wl.T, wl.H, wl.I, wl.E, wl.k, wl.wdtype, "auto")
+    shape = moe.make_shape(wl.T, wl.H, wl.I, wl.E, wl.k, wl.wdtype, args.path)
     lay = moe.workspace_layout(shape)
     path = moe.PATH_NAMES[lay.path]
     stream = torch.cuda.current_stream()
@@ -484,8 +509,9 @@ def measure(moe, wl, args, world, rank, local, peaks, peak_src):
         router_line = time_router(moe, wl, seed, xd, flush, stream, K, args.warmup, world, peaks)
 
     # route, permute, gate/up, down, combine; the e4m3 DECODE path adds the
-    # per-token x quantisation and the h quantisation
-    per_step_launches = (1 + (1 if wl.T <= 256 else 3) + 2 + 1
+    # per-token x quantisation and the h quantisation; FUSED is route + one kernel
+    per_step_launches = (2 if path == "fused" else
+                         1 + (1 if wl.T <= 256 else 3) + 2 + 1
                          + (2 if path == "decode" and wl.wdtype == "e4m3" else 0))
     tokens = wl.T * K * world
     line = {
@@ -545,6 +571,8 @@ def main():
     ap.add_argument("--workload", choices=list(G.WORKLOADS), default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", action="store_true", help="measure the chosen workload alone (no per_config)")
+    ap.add_argument("--path", choices=["auto", "prefill", "decode", "fused"], default="auto",
+                    help="execution path of every measured layer (default: the library's choice)")
     ap.add_argument("--router", action="store_true",
                     help="also time the fused router (router GEMM + top-k) on the workload's tokens")
     ap.add_argument("--shape", default=None,

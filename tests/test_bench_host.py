@@ -73,6 +73,12 @@ def test_roofline_arithmetic():
     byts = 90 * 2 * wl.I * wl.H + 90 * (2 * wl.I // 128) * (wl.H // 128) + wl.T * wl.H * 2 + wl.A * wl.I
     assert r["kernel"] == "decode_e4m3_gate_up_kernel"
     assert abs(r["achieved"] - byts / 5e-4 / 1e9) < 1e-6 * r["achieved"]
+    # the fused path: one kernel streams every touched expert's three matrices
+    wl = G.WORKLOADS["decode"]
+    r = bench.stage_roofline(wl, "fused", {1: 0.15, 2: 0.0}, 42, peaks, "measured")
+    byts = 42 * 3 * wl.I * wl.H * 2 + 2 * wl.T * wl.H * 2
+    assert r["kernel"] == "fused_decode_kernel" and r["bound"] == "hbm"
+    assert abs(r["achieved"] - byts / 1.5e-4 / 1e9) < 1e-6 * r["achieved"]
 
 
 def test_reference_arm_runs_on_cpu():
