@@ -107,6 +107,17 @@ def oracle_forward_fp8(x_cpu, idx, w, W, tokens=None, cache=True):
                              ExpertView(W["sw_down"], True, cache), tokens=tokens)
 
 
+def device_topk_w(logits_cpu, k, idx_ref):
+    """The routing weights the device itself uses for these logits (moe_route
+    is deterministic, so a layer that routed the same logits got these bits),
+    after checking that its indices equal the oracle's. The combine pin takes
+    these: the device's weights differ from the oracle's by exp/division
+    rounding, which a bit-exact comparison must not see."""
+    idx_d, w_d = moe.route(logits_cpu.cuda(), k)
+    assert np.array_equal(idx_d.cpu().numpy(), idx_ref)
+    return w_d.cpu().numpy()
+
+
 def check_combine_bit_exact(ws, shape, topk_w_np, out, chunk=1024):
     """The device combine against the oracle's fixed-order fp32 combine on the
     expert outputs y the device itself produced (read from the workspace):

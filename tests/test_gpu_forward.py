@@ -11,7 +11,7 @@ from mixture_experts_routed_moe_b200 import inputs as G
 from oracle import moe_oracle as O
 
 from parity import (ExpertView, assert_bf16_close, assert_tokens_close, check_combine_bit_exact,
-                    check_permutation, device_inputs, oracle_forward_bf16, ws_bf16)
+                    check_permutation, device_inputs, device_topk_w, oracle_forward_bf16, ws_bf16)
 
 pytestmark = pytest.mark.gpu
 
@@ -181,7 +181,7 @@ def test_full_size_bf16_every_token(name):
     assert moe.read_device_status(ws) == 0
     shape = moe.make_shape(wl.T, wl.H, wl.I, wl.E, wl.k, "bf16", "auto")
     lay, perm = check_permutation(ws, shape, idx)
-    check_combine_bit_exact(ws, shape, w, out)
+    check_combine_bit_exact(ws, shape, device_topk_w(L, wl.k, idx), out)
     _expert_block_check(ws, lay, perm, x, idx, W, wl, [0, wl.E // 2, wl.E - 1])
     ref = oracle_forward_bf16(x, idx, w, W, cache=False)
     got = out.float().cpu().numpy()

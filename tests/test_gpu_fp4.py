@@ -12,7 +12,7 @@ import mixture_experts_routed_moe_b200 as moe
 from mixture_experts_routed_moe_b200 import inputs as G
 from oracle import moe_oracle as O
 
-from parity import (ExpertView, assert_bf16_close, assert_tokens_close, check_combine_bit_exact, check_permutation,
+from parity import (ExpertView, assert_bf16_close, assert_tokens_close, check_combine_bit_exact, check_permutation, device_topk_w,
                     device_inputs, ws_bf16)
 
 pytestmark = pytest.mark.gpu
@@ -84,7 +84,7 @@ def test_fp4_decode_full_size_every_token():
     assert moe.workspace_layout(shape).path == moe.PATH["decode"]
     idx, w, _ = O.route(L.numpy(), wl.k)
     check_permutation(ws, shape, idx)
-    check_combine_bit_exact(ws, shape, w, out)
+    check_combine_bit_exact(ws, shape, device_topk_w(L, wl.k, idx), out)
     ref = oracle_fp4(x, idx, w, W, cache=False)
     got = out.float().cpu().numpy()
     assert_bf16_close(got, ref, "fp4 decode full")
@@ -149,7 +149,7 @@ def test_fp4_full_size_every_token():
     assert moe.workspace_layout(shape).path == moe.PATH["prefill"]
     idx, w, _ = O.route(L.numpy(), wl.k)
     check_permutation(ws, shape, idx)
-    check_combine_bit_exact(ws, shape, w, out)
+    check_combine_bit_exact(ws, shape, device_topk_w(L, wl.k, idx), out)
     ref = oracle_fp4(x, idx, w, W, cache=False)
     got = out.float().cpu().numpy()
     assert_bf16_close(got, ref, "fp4 full")

@@ -10,7 +10,7 @@ import mixture_experts_routed_moe_b200 as moe
 from mixture_experts_routed_moe_b200 import inputs as G
 from oracle import moe_oracle as O
 
-from parity import (ExpertView, assert_fp8_close, assert_tokens_close, check_combine_bit_exact, check_permutation,
+from parity import (ExpertView, assert_fp8_close, assert_tokens_close, check_combine_bit_exact, check_permutation, device_topk_w,
                     device_inputs, oracle_forward_fp8, rel_fro)
 
 # Per-token bound for FP8 layers: the layer's stated bound (3e-2 relative
@@ -112,7 +112,7 @@ def test_fp8_decode_full_size_every_token():
     assert moe.workspace_layout(shape).path == moe.PATH["decode"]
     idx, w, _ = O.route(L.numpy(), wl.k)
     check_permutation(ws, shape, idx)
-    check_combine_bit_exact(ws, shape, w, out)
+    check_combine_bit_exact(ws, shape, device_topk_w(L, wl.k, idx), out)
     ref = oracle_forward_fp8(x, idx, w, W, cache=False)
     got = out.float().cpu().numpy()
     assert assert_fp8_close(got, ref, "fp8 decode full") < 1e-2
@@ -154,7 +154,7 @@ def test_fp8_full_size_every_token():
     idx, w, _ = O.route(L.numpy(), wl.k)
     shape = moe.make_shape(wl.T, wl.H, wl.I, wl.E, wl.k, "e4m3")
     lay, perm = check_permutation(ws, shape, idx)
-    check_combine_bit_exact(ws, shape, w, out)
+    check_combine_bit_exact(ws, shape, device_topk_w(L, wl.k, idx), out)
     # x codes and scales: quantised once per token by the oracle, compared on every permuted row
     codes, scales, xdq = O.quantize_1x128(x.float().numpy())
     rows = np.nonzero(perm["row_src"] >= 0)[0]
