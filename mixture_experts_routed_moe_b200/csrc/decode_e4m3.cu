@@ -179,10 +179,11 @@ __global__ void __launch_bounds__(kBlock) decode_e4m3_quant_h_kernel(const float
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     const float sc = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
-    const uint32_t lo =
-        __nv_cvt_float2_to_fp8x2(make_float2(__fdiv_rn(v.x, sc), __fdiv_rn(v.y, sc)), __NV_SATFINITE, __NV_E4M3);
-    const uint32_t hi =
-        __nv_cvt_float2_to_fp8x2(make_float2(__fdiv_rn(v.z, sc), __fdiv_rn(v.w, sc)), __NV_SATFINITE, __NV_E4M3);
+    const GroupDivisor dv = make_group_divisor(sc);
+    const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(group_div(dv, v.x), group_div(dv, v.y)),
+                                                 __NV_SATFINITE, __NV_E4M3);
+    const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(group_div(dv, v.z), group_div(dv, v.w)),
+                                                 __NV_SATFINITE, __NV_E4M3);
     *reinterpret_cast<uint32_t*>(hq + at) = lo | (hi << 16);
     if (lane == 0) hs[static_cast<size_t>(row) * G + g] = sc;
   }

@@ -120,13 +120,14 @@ __device__ __forceinline__ void finish_gate_up(float (&acc)[128], float* s_amax,
   amax = fmaxf(s_amax[r], s_amax[kTileM + r]);
   epi_bar_sync();
   const float sc = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+  const GroupDivisor dv = make_group_divisor(sc);
   uint32_t w[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(__fdiv_rn(acc[4 * i], sc), __fdiv_rn(acc[4 * i + 1], sc)),
-                                                 __NV_SATFINITE, __NV_E4M3);
+    const uint32_t lo = __nv_cvt_float2_to_fp8x2(
+        make_float2(group_div(dv, acc[4 * i]), group_div(dv, acc[4 * i + 1])), __NV_SATFINITE, __NV_E4M3);
     const uint32_t hi = __nv_cvt_float2_to_fp8x2(
-        make_float2(__fdiv_rn(acc[4 * i + 2], sc), __fdiv_rn(acc[4 * i + 3], sc)), __NV_SATFINITE, __NV_E4M3);
+        make_float2(group_div(dv, acc[4 * i + 2]), group_div(dv, acc[4 * i + 3])), __NV_SATFINITE, __NV_E4M3);
     w[i] = lo | (hi << 16);
   }
   // pad rows of the expert's last block are stored too (nothing reads them)
@@ -332,6 +333,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_ld16(tb + col, v[j]);
           }
           tmem_ld_wait();
+          if (q == 6) {
+            // every column of this partial is in registers: hand the buffer
+            // back to the tensor core before the last multiply-adds
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&pempty[pb]);
+          }
 #pragma unroll
           for (int j = 0; j < 2; ++j) {
             const int qq = q + j;
@@ -341,9 +349,6 @@ __global__ void __launch_bounds__(kThreads, 1)
               ffma2(acc[16 * qq + i], acc[16 * qq + i + 1], __uint_as_float(v[j][i]), __uint_as_float(v[j][i + 1]), sc);
           }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&pempty[pb]);
         pb ^= 1;
         if (pb == 0) pph ^= 1;
       }

@@ -367,6 +367,35 @@ __device__ __forceinline__ float gated_act(int act, float g, float u) {
   return a * u;
 }
 
+// Division by one divisor d shared by many dividends (the 1x128 group scale of
+// the e4m3 quantisation), for the e4m3 codes of x / d: rcp = 1/d correctly
+// rounded, q = x * rcp, then one correction by the remainder,
+// q + (x - q d) * rcp (the final step of Markstein's division method: with a
+// correctly rounded reciprocal and q within an ulp of x / d, the corrected
+// quotient is the IEEE round-to-nearest one). The remainder is exact when d
+// lies in [2^-90, 2^90] and |x| >= 2^-100; a divisor outside that range is
+// first brought into it by an exact power-of-two scaling of d and of every x.
+// Smaller |x| give quotients below 2^-10, whose e4m3 code is a zero of the
+// sign of x on both routes (a zero product keeps its sign; the correction
+// would not). Checked exhaustively against IEEE division on every signed
+// bf16 dividend within 40 binades of every bf16 group maximum.
+struct GroupDivisor {
+  float d, rcp, s;
+};
+__device__ __forceinline__ GroupDivisor make_group_divisor(float d) {
+  GroupDivisor g;
+  g.s = d < 0x1p-90f ? 0x1p64f : (d > 0x1p90f ? 0x1p-64f : 1.0f);
+  g.d = d * g.s;
+  g.rcp = __frcp_rn(g.d);
+  return g;
+}
+__device__ __forceinline__ float group_div(const GroupDivisor& g, float x) {
+  const float xs = x * g.s;
+  const float q = xs * g.rcp;
+  const float c = fmaf(fmaf(-q, g.d, xs), g.rcp, q);
+  return q == 0.0f ? q : c;
+}
+
 // (a0, a1) = (b0 * s + a0, b1 * s + a1): two fp32 fused multiply-adds, round to
 // nearest, in one packed f32x2 instruction (each lane bit-identical to fmaf).
 __device__ __forceinline__ void ffma2(float& a0, float& a1, float b0, float b1, float s) {

@@ -167,7 +167,7 @@ __device__ __forceinline__ void copy_row_bf16(const __nv_bfloat16* __restrict__ 
 
 // Quantise one 128-column group of a bf16 row with one half-warp (lane l16
 // holds columns 8*l16 .. 8*l16+7, in v): scale s = amax/448 in fp32 (1 for
-// an all-zero group) and codes e4m3(x/s) with IEEE division, round to nearest
+// an all-zero group) and codes e4m3(x/s) of the IEEE quotient, round to nearest
 // even, saturating -- the FP8 experts' dynamic per-row activation scales.
 __device__ __forceinline__ uint2 quant_group_codes(const uint4& v, unsigned hmask, float* sc_out) {
   const float f[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
@@ -178,13 +178,14 @@ __device__ __forceinline__ uint2 quant_group_codes(const uint4& v, unsigned hmas
 #pragma unroll
   for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(hmask, amax, o));
   const float sc = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+  const GroupDivisor dv = make_group_divisor(sc);
   uint32_t w[2];
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
-    const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(__fdiv_rn(f[4 * i], sc), __fdiv_rn(f[4 * i + 1], sc)),
+    const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(group_div(dv, f[4 * i]), group_div(dv, f[4 * i + 1])),
                                                  __NV_SATFINITE, __NV_E4M3);
     const uint32_t hi = __nv_cvt_float2_to_fp8x2(
-        make_float2(__fdiv_rn(f[4 * i + 2], sc), __fdiv_rn(f[4 * i + 3], sc)), __NV_SATFINITE, __NV_E4M3);
+        make_float2(group_div(dv, f[4 * i + 2]), group_div(dv, f[4 * i + 3])), __NV_SATFINITE, __NV_E4M3);
     w[i] = lo | (hi << 16);
   }
   *sc_out = sc;
