@@ -33,31 +33,39 @@ __device__ __forceinline__ float route_key_value(uint32_t key) {
 // row: the token's E logits (global or shared memory); idx_out / w_out: its k slots.
 template <int kPerLane>
 __device__ __forceinline__ void route_token(const float* row, int E, int k, int lane, int* idx_out, float* w_out) {
-  float v[kPerLane];
+  // keys of this lane's logits (expert lane + 32*i); a taken or absent expert
+  // has key 0, below every logit's key
+  uint32_t key[kPerLane];
 #pragma unroll
   for (int i = 0; i < kPerLane; ++i) {
     const int e = lane + 32 * i;
-    v[i] = (e < E) ? row[e] : -INFINITY;
+    key[i] = (e < E) ? route_key(row[e]) : 0u;
   }
-  uint32_t taken = 0;  // bit i: expert lane + 32*i already selected
   float vmax = 0.f, psum = 0.f, pcomp = 0.f;
+  // slot j < 32 is kept by lane j until the end (the k selected experts and
+  // their softmax numerators), so the slots are written once, coalesced
+  int my_idx = 0;
+  float my_p = 0.f;
   for (int j = 0; j < k; ++j) {
     // this lane's best untaken expert (i ascending keeps the lower index on ties)
-    uint32_t key = 0;  // below every logit's key: no candidate
-    int bi = 0x7fffffff;
+    uint32_t best = 0;
+    int bi = 0;
 #pragma unroll
     for (int i = 0; i < kPerLane; ++i) {
-      const int e = lane + 32 * i;
-      const uint32_t ki = route_key(v[i]);
-      if (e < E && !(taken & (1u << i)) && (ki > key || bi == 0x7fffffff)) {
-        key = ki;
-        bi = e;
+      if (key[i] > best) {
+        best = key[i];
+        bi = i;
       }
     }
-    const uint32_t kmax = __reduce_max_sync(0xffffffffu, key);
-    const int win = static_cast<int>(
-        __reduce_min_sync(0xffffffffu, key == kmax ? static_cast<uint32_t>(bi) : 0x7fffffffu));
-    if ((win & 31) == lane) taken |= 1u << (win >> 5);
+    const uint32_t kmax = __reduce_max_sync(0xffffffffu, best);
+    // lanes holding the maximum offer their expert; the lowest index wins
+    const uint32_t cand = (best == kmax && kmax != 0u) ? static_cast<uint32_t>(lane + 32 * bi) : 0x7fffffffu;
+    const int win = static_cast<int>(__reduce_min_sync(0xffffffffu, cand));
+    if ((win & 31) == lane) {
+#pragma unroll
+      for (int i = 0; i < kPerLane; ++i)
+        if (i == (win >> 5)) key[i] = 0u;
+    }
     const float bv = route_key_value(kmax);
     if (j == 0) vmax = bv;
     const float p = expf(bv - vmax);  // exp(l_j - l_max): the softmax numerator
@@ -65,14 +73,25 @@ __device__ __forceinline__ void route_token(const float* row, int E, int k, int 
     const float tk = psum + yk;
     pcomp = (tk - psum) - yk;
     psum = tk;
-    if (lane == 0) {
+    if (j < 32) {
+      if (lane == j) {
+        my_idx = win;
+        my_p = p;
+      }
+    } else if (lane == 0) {  // slots beyond 32 go out now and are rescaled below
       idx_out[j] = win;
       w_out[j] = p;
     }
   }
-  __syncwarp();
-  // renormalise over the chosen k (each lane rescales its own slots)
-  for (int j = lane; j < k; j += 32) w_out[j] = w_out[j] / psum;
+  // renormalise over the chosen k
+  if (lane < k) {
+    idx_out[lane] = my_idx;
+    w_out[lane] = my_p / psum;
+  }
+  if (k > 32) {
+    __syncwarp();
+    for (int j = 32 + lane; j < k; j += 32) w_out[j] = w_out[j] / psum;
+  }
 }
 
 }  // namespace moe
