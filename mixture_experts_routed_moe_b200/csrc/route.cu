@@ -4,7 +4,7 @@
 //
 // One warp per token over logits in global memory; the per-token selection
 // (fp32 softmax denominator, k shuffle arg-max rounds with ties to the lower
-// index, compensated renormalisation) is route_token in route_core.cuh.
+// index, renormalisation over the chosen k) is route_token in route_core.cuh.
 #include "moe_common.cuh"
 #include "moe_internal.h"
 #include "route_core.cuh"

@@ -13,7 +13,8 @@
 // The weights are the softmax probabilities renormalised over the k chosen
 // experts: w_j = exp(l_j - l_max) / sum_j' exp(l_j' - l_max), where the first
 // selected logit is l_max and the softmax denominator over all E experts
-// cancels. The sum is compensated (Kahan).
+// cancels. The k numerators are computed after the selection, one per lane,
+// and summed in a fixed butterfly order.
 #pragma once
 
 #include "moe_common.cuh"
@@ -41,11 +42,11 @@ __device__ __forceinline__ void route_token(const float* row, int E, int k, int 
     const int e = lane + 32 * i;
     key[i] = (e < E) ? route_key(row[e]) : 0u;
   }
-  float vmax = 0.f, psum = 0.f, pcomp = 0.f;
-  // slot j < 32 is kept by lane j until the end (the k selected experts and
-  // their softmax numerators), so the slots are written once, coalesced
+  // selection: slot j < 32 is kept by lane j (its expert and key); later
+  // slots (k > 32) go to global memory at once
   int my_idx = 0;
-  float my_p = 0.f;
+  uint32_t my_key = 0;
+  uint32_t key0 = 0;
   for (int j = 0; j < k; ++j) {
     // this lane's best untaken expert (i ascending keeps the lower index on ties)
     uint32_t best = 0;
@@ -66,31 +67,43 @@ __device__ __forceinline__ void route_token(const float* row, int E, int k, int 
       for (int i = 0; i < kPerLane; ++i)
         if (i == (win >> 5)) key[i] = 0u;
     }
-    const float bv = route_key_value(kmax);
-    if (j == 0) vmax = bv;
-    const float p = expf(bv - vmax);  // exp(l_j - l_max): the softmax numerator
-    const float yk = p - pcomp;
-    const float tk = psum + yk;
-    pcomp = (tk - psum) - yk;
-    psum = tk;
+    if (j == 0) key0 = kmax;
     if (j < 32) {
       if (lane == j) {
         my_idx = win;
-        my_p = p;
+        my_key = kmax;
       }
-    } else if (lane == 0) {  // slots beyond 32 go out now and are rescaled below
+    } else if (lane == 0) {
       idx_out[j] = win;
-      w_out[j] = p;
+      w_out[j] = route_key_value(kmax);  // the logit for now; the weight below
     }
   }
-  // renormalise over the chosen k
+  // weights: the softmax numerators exp(l_j - l_max) of the chosen experts,
+  // one per lane, their sum over the k slots (a fixed butterfly order, and
+  // for k > 32 the later slots added in slot order, compensated), and p_j / sum
+  const float vmax = route_key_value(key0);
+  const float p = lane < k ? expf(route_key_value(my_key) - vmax) : 0.f;
+  float psum = p;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) psum += __shfl_xor_sync(0xffffffffu, psum, o);
+  if (k > 32) {
+    // the later slots' numerators, added in slot order with compensation (Kahan)
+    __syncwarp();
+    float rest = 0.f, comp = 0.f;
+    for (int j = 32; j < k; ++j) {
+      const float yk = expf(w_out[j] - vmax) - comp;
+      const float tk = rest + yk;
+      comp = (tk - rest) - yk;
+      rest = tk;
+    }
+    psum += rest;
+    __syncwarp();
+    if (lane == 0)
+      for (int j = 32; j < k; ++j) w_out[j] = expf(w_out[j] - vmax) / psum;
+  }
   if (lane < k) {
     idx_out[lane] = my_idx;
-    w_out[lane] = my_p / psum;
-  }
-  if (k > 32) {
-    __syncwarp();
-    for (int j = 32 + lane; j < k; j += 32) w_out[j] = w_out[j] / psum;
+    w_out[lane] = p / psum;
   }
 }
 
