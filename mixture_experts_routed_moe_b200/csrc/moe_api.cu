@@ -105,10 +105,16 @@ bool validate_shape(const moe_shape* s) {
   return true;
 }
 
+// Decode-stage switch: the weight-streaming path while the assignments per
+// expert stay at or below the crossover with the grouped GEMMs measured on
+// B200 (sweeps of T on the decode- and large-layer shapes): two per expert
+// for bf16 and FP4 experts, one half for e4m3 experts, whose streaming path
+// widens codes on the CUDA cores.
 int resolve_path(const moe_shape* s) {
   if (s->path != MOE_PATH_AUTO) return s->path;
-  if (static_cast<long long>(s->T) * s->k <= 4ll * s->E && decode_supported(s))
-    return MOE_PATH_DECODE;
+  const long long A = static_cast<long long>(s->T) * s->k;
+  const bool small = s->wdtype == MOE_DT_E4M3 ? 2 * A <= s->E : A <= 2ll * s->E;
+  if (small && decode_supported(s)) return MOE_PATH_DECODE;
   return MOE_PATH_PREFILL;
 }
 

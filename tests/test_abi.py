@@ -106,10 +106,18 @@ def test_e4m3_workspace_layouts(L):
 
 
 def test_auto_path_choice(L):
-    assert moe.workspace_layout(shape(T=16, H=2048, I=1408, E=60, k=4)).path == moe.PATH["decode"]
-    assert moe.workspace_layout(shape(T=8192, H=2048, I=768, E=128, k=8)).path == moe.PATH["prefill"]
-    assert moe.workspace_layout(shape(T=16, E=60, k=4, wdtype="e4m3")).path == moe.PATH["decode"]
-    assert moe.workspace_layout(shape(T=4096, E=60, k=4, wdtype="e4m3")).path == moe.PATH["prefill"]
+    """The decode-stage switch: streaming while T*k <= 2E (bf16, FP4) or
+    2*T*k <= E (e4m3), the grouped GEMMs beyond; the boundary cases included."""
+    D, P = moe.PATH["decode"], moe.PATH["prefill"]
+    assert moe.workspace_layout(shape(T=16, H=2048, I=1408, E=60, k=4)).path == D
+    assert moe.workspace_layout(shape(T=30, H=2048, I=1408, E=60, k=4)).path == D  # 120 = 2E
+    assert moe.workspace_layout(shape(T=31, H=2048, I=1408, E=60, k=4)).path == P
+    assert moe.workspace_layout(shape(T=8192, H=2048, I=768, E=128, k=8)).path == P
+    assert moe.workspace_layout(shape(T=16, H=7168, I=2048, E=256, k=8, wdtype="e4m3")).path == D  # 128 = E/2
+    assert moe.workspace_layout(shape(T=17, H=7168, I=2048, E=256, k=8, wdtype="e4m3")).path == P
+    assert moe.workspace_layout(shape(T=64, H=7168, I=2048, E=256, k=8, wdtype="e2m1")).path == D  # 512 = 2E
+    assert moe.workspace_layout(shape(T=65, H=7168, I=2048, E=256, k=8, wdtype="e2m1")).path == P
+    assert moe.workspace_layout(shape(T=4096, E=60, k=4, wdtype="e4m3")).path == P
 
 
 def test_scale_format_error_and_host_errors(L):
