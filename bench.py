@@ -63,7 +63,7 @@ FLUSH_BYTES = 256 << 20
 # unchanged (first 16 hex digits of the .cu file's SHA-256). "scaled" says how
 # a capture of a smaller case was brought to one full launch.
 NCU_TRAFFIC = {
-    ("decode", "decode_gate_up_kernel"): {"bytes": 488657920, "src": "003fad137931ac74", "scaled": None},
+    ("decode", "small_gemm_bf16_kernel<true>"): {"bytes": 488641280, "src": "a3bfce7023d13b12", "scaled": None},
     ("prefill", "grouped_gemm_bf16_kernel<256,true>"): {"bytes": 1211534704, "src": "d64f0e084cc41143",
                                                          "scaled": None},
     ("fp8", "grouped_gemm_e4m3_kernel<true>"): {"bytes": 8316361440, "src": "dc4eb5e6a4256cd9",
@@ -308,12 +308,12 @@ def stage_roofline(wl, path, stage_ms, n_touched, peaks, peak_src):
             byts = int(n_touched * 2 * I * H * welem) + s_gu + wl.T * H * 2 + h_bytes
             kern, src = (("decode_e4m3_gate_up_kernel", "decode_e4m3.cu") if fp8 else
                          ("decode_fp4_gate_up_kernel", "decode_fp4.cu") if fp4 else
-                         ("decode_gate_up_kernel", "decode.cu"))
+                         ("small_gemm_bf16_kernel<true>", "gemm_small.cu"))
         else:
             byts = int(n_touched * H * I * welem) + s_d + h_bytes + A * H * 2
             kern, src = (("decode_e4m3_down_kernel", "decode_e4m3.cu") if fp8 else
                          ("decode_fp4_down_kernel", "decode_fp4.cu") if fp4 else
-                         ("decode_down_kernel", "decode.cu"))
+                         ("small_gemm_bf16_kernel<false>", "gemm_small.cu"))
         ach = byts / dur_s / 1e9
         peak = peaks["hbm_gbs"]
         out = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
@@ -508,9 +508,17 @@ def measure(moe, wl, args, world, rank, local, peaks, peak_src):
 
     # route, permute, gate/up, down, combine; the e4m3 DECODE path adds the
     # per-token x quantisation and the h quantisation; FUSED is route + one kernel
+    # route, permute (one kernel up to 256 tokens, else three) plus a row-staging
+    # kernel where the single-block permute does not copy the rows itself
+    # (more than 32768 elements to copy, or the e4m3 DECODE path's per-token
+    # quantisation), gate/up, down (and the e4m3 DECODE path's h quantisation),
+    # combine; FUSED is route + one kernel
+    copies_rows = path == "prefill" or (path == "decode" and wl.wdtype == "bf16")
+    stage_launch = ((wl.T <= 256 and copies_rows and wl.A * wl.H > 32768)
+                    or (path == "decode" and wl.wdtype == "e4m3"))
     per_step_launches = (2 if path == "fused" else
-                         1 + (1 if wl.T <= 256 else 3) + 2 + 1
-                         + (2 if path == "decode" and wl.wdtype == "e4m3" else 0))
+                         1 + (1 if wl.T <= 256 else 3) + int(stage_launch) + 2 + 1
+                         + (1 if path == "decode" and wl.wdtype == "e4m3" else 0))
     tokens = wl.T * K * world
     line = {
         "value": tokens / (total_ms / 1e3), "unit": "tokens/s", "ms_per_step": total_ms / K,

@@ -58,7 +58,7 @@ typedef enum {
 /* Which execution of the expert matmuls to use (the page's decode-stage switch:
  * small token counts run better on a per-token form than on grouped GEMM tiles). */
 typedef enum {
-  MOE_PATH_AUTO = 0,    /* DECODE when T*k <= 2*E (e4m3 experts: 2*T*k <= E), else PREFILL */
+  MOE_PATH_AUTO = 0,    /* DECODE when T*k <= 32*E (bf16), 2*E (e2m1), E/2 (e4m3); else PREFILL */
   MOE_PATH_PREFILL = 1, /* expert-major permute + tcgen05 grouped GEMMs */
   MOE_PATH_DECODE = 2,  /* weight-streaming kernels, no tile padding */
   MOE_PATH_FUSED = 3    /* the DECODE path's permute, gate/up, down and combine in one

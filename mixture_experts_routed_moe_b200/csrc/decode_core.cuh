@@ -1,9 +1,10 @@
-// Weight-streaming building blocks of the small-token expert forward, shared by
-// the decode kernels (decode.cu) and the fused single-launch forward
-// (fused_decode.cu). With only a few tokens per expert the layer is bound by
-// reading each touched expert's weights once from HBM: a warp owns a few
-// consecutive weight rows of one expert, streams them with 16-byte no-L1 loads
-// and dots them against up to four of that expert's activation rows.
+// Weight-streaming building blocks of the small-token expert forward on the
+// CUDA cores, used by the fused single-launch forward (fused_decode.cu) and
+// the FP4 decode kernels (decode_fp4.cu). With only a few tokens per expert
+// the layer is bound by reading each touched expert's weights once from HBM:
+// a warp owns a few consecutive weight rows of one expert, streams them with
+// 16-byte no-L1 loads and dots them against up to four of that expert's
+// activation rows.
 #pragma once
 
 #include "moe_common.cuh"

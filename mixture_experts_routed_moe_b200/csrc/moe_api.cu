@@ -105,16 +105,19 @@ bool validate_shape(const moe_shape* s) {
   return true;
 }
 
-// Decode-stage switch: the weight-streaming path while the assignments per
-// expert stay at or below the crossover with the grouped GEMMs measured on
-// B200 (sweeps of T on the decode- and large-layer shapes): two per expert
-// for bf16 and FP4 experts, one half for e4m3 experts, whose streaming path
-// widens codes on the CUDA cores.
+// Decode-stage switch: the DECODE path while the assignments per expert stay
+// at or below the crossover with the grouped GEMMs measured on B200 (sweeps
+// of T on the decode- and large-layer shapes): 32 per expert for bf16
+// experts (tensor-core GEMMs with the tokens as N, which stream the weights
+// at HBM rate up to 128 tokens per expert), two for FP4 experts and one half
+// for e4m3 experts, whose DECODE kernels widen codes on the CUDA cores.
 int resolve_path(const moe_shape* s) {
   if (s->path != MOE_PATH_AUTO) return s->path;
   const long long A = static_cast<long long>(s->T) * s->k;
-  const bool small = s->wdtype == MOE_DT_E4M3 ? 2 * A <= s->E : A <= 2ll * s->E;
-  if (small && decode_supported(s)) return MOE_PATH_DECODE;
+  const bool small = s->wdtype == MOE_DT_E4M3   ? 2 * A <= s->E
+                     : s->wdtype == MOE_DT_E2M1 ? A <= 2ll * s->E
+                                                : A <= 32ll * s->E;
+  if (small) return MOE_PATH_DECODE;
   return MOE_PATH_PREFILL;
 }
 
@@ -157,7 +160,8 @@ bool make_plan(const moe_shape* s, Plan* p) {
   // bf16 DECODE reads the token rows of x in place
   // (e4m3 DECODE: one row per token, not per assignment)
   const size_t xrows = (fp8 && streaming) ? static_cast<size_t>(T) : M;
-  p->xa = (p->path == MOE_PATH_PREFILL || fp8) ? take(xrows * H * act) : none;
+  p->tc_stream = p->path == MOE_PATH_DECODE && small_gemm_supported(s);
+  p->xa = (p->path == MOE_PATH_PREFILL || fp8 || p->tc_stream) ? take(xrows * H * act) : none;
   p->xs = fp8 ? take(xrows * (H / 128) * 4) : none;
   p->h = take(M * I * act);
   p->hs = fp8 ? take(M * (I / 128) * 4) : none;
@@ -237,7 +241,6 @@ moe_status forward_impl(const moe_shape* shape, const void* x, const int32_t* to
   // e4m3 PREFILL: the down tile spans two 128-column scale blocks
   if (fp8 && plan.path == MOE_PATH_PREFILL && (!e4m3_path_available() || shape->H % 256 != 0))
     return MOE_ERR_UNSUPPORTED;
-  if (plan.path == MOE_PATH_DECODE && !decode_supported(shape)) return MOE_ERR_UNSUPPORTED;
   if (plan.path == MOE_PATH_FUSED && !fused_supported(shape)) return MOE_ERR_UNSUPPORTED;
   if (shape->T == 0) return MOE_OK;
   if (x == nullptr || topk_idx == nullptr || topk_w == nullptr || w_gate_up == nullptr || w_down == nullptr ||
@@ -276,9 +279,9 @@ moe_status forward_impl(const moe_shape* shape, const void* x, const int32_t* to
     if (err != cudaSuccess || !mark(2)) return MOE_ERR_CUDA;
     err = launch_decode_e4m3(shape, plan, w_gate_up, w_down, sw_gate_up, sw_down, ws, 1, sms, st);
   } else if (plan.path == MOE_PATH_DECODE) {
-    err = launch_decode(shape, plan, x, w_gate_up, w_down, ws, 0, sms, st);
+    err = launch_small_gemm(shape, plan, w_gate_up, w_down, ws, 0, sms, st);
     if (err != cudaSuccess || !mark(2)) return MOE_ERR_CUDA;
-    err = launch_decode(shape, plan, x, w_gate_up, w_down, ws, 1, sms, st);
+    err = launch_small_gemm(shape, plan, w_gate_up, w_down, ws, 1, sms, st);
   } else if (fp4) {
     err = launch_gemm_fp4(shape, plan, w_gate_up, w_down, sw_gate_up, sw_down, ws, 0, sms, st);
     if (err != cudaSuccess || !mark(2)) return MOE_ERR_CUDA;

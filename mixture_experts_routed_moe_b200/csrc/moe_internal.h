@@ -34,6 +34,7 @@ struct Plan {
   size_t status, hdr, block_counts, cnt, mt_base, pt_base, touched, local_rank, row_src, slot_row;
   size_t sync;  // FUSED path: task queues and per-expert completion counters (3 + 2E ints)
   size_t xa, xs, h, hs, hf, y, total;  // hf: fp32 h of the e4m3 DECODE path
+  bool tc_stream;  // bf16 DECODE: tensor-core GEMMs with the tokens as N, x rows staged into xa
 };
 
 // Words of the status block (workspace offset `status`), all zeroed by the
@@ -72,9 +73,11 @@ cudaError_t launch_gemm_e4m3(const moe_shape* s, const Plan& p, const void* x, c
                              int which, int num_sms, cudaStream_t st);
 bool e4m3_path_available();
 
-bool decode_supported(const moe_shape* s);
-cudaError_t launch_decode(const moe_shape* s, const Plan& p, const void* x, const void* w_gate_up,
-                          const void* w_down, uint8_t* ws, int which, int num_sms, cudaStream_t st);
+// bf16 experts on the DECODE path with the expert's token rows as the MMA's N
+// (which = 0 gate/up from the staged x rows, 1 down).
+bool small_gemm_supported(const moe_shape* s);
+cudaError_t launch_small_gemm(const moe_shape* s, const Plan& p, const void* w_gate_up, const void* w_down,
+                              uint8_t* ws, int which, int num_sms, cudaStream_t st);
 // e4m3 experts on the DECODE path: which = 0 runs gate/up and the h
 // quantisation, which = 1 the down projection.
 cudaError_t launch_decode_e4m3(const moe_shape* s, const Plan& p, const void* w_gate_up, const void* w_down,

@@ -409,8 +409,10 @@ cudaError_t launch_permute(const moe_shape* s, const Plan& p, const int* topk_id
   const bool fp8 = s->wdtype == MOE_DT_E4M3;
   const bool prefill = p.path == MOE_PATH_PREFILL;
   // PREFILL: x copied (bf16) or quantised (e4m3) into the permuted rows;
-  // e4m3 DECODE: x quantised once per token; bf16 DECODE reads x in place
-  __nv_bfloat16* xa = (prefill && !fp8) ? reinterpret_cast<__nv_bfloat16*>(ws + p.xa) : nullptr;
+  // e4m3 DECODE: x quantised once per token; bf16 DECODE: x copied into the
+  // expert-major rows for the tensor-core kernels, else read in place
+  const bool copy_x = (prefill || p.tc_stream) && !fp8;
+  __nv_bfloat16* xa = copy_x ? reinterpret_cast<__nv_bfloat16*>(ws + p.xa) : nullptr;
   uint8_t* xq = fp8 ? ws + p.xa : nullptr;
   float* xs = fp8 ? reinterpret_cast<float*>(ws + p.xs) : nullptr;
   const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
@@ -419,7 +421,7 @@ cudaError_t launch_permute(const moe_shape* s, const Plan& p, const int* topk_id
   const int G = H / 128;
   // rows are staged by the permute kernels themselves only where that is
   // short: the single-block permute for at most kSmallStageElems elements
-  const bool stage_in_small = prefill && A * H <= kSmallStageElems;
+  const bool stage_in_small = (prefill || copy_x) && A * H <= kSmallStageElems;
   auto stage = [&](const int* slots, long long n_src) -> cudaError_t {
     const long long tasks = n_src * G;
     const long long want = (tasks + 15) / 16;  // blocks of 16 half-warps
@@ -438,8 +440,8 @@ cudaError_t launch_permute(const moe_shape* s, const Plan& p, const int* topk_id
                                                       stage_in_small ? xq : nullptr,
                                                       stage_in_small ? xs : nullptr, H);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
-    if (stage_in_small || (!prefill && !fp8)) return cudaSuccess;
-    return prefill ? stage(slot_row, A) : stage(nullptr, T);
+    if (stage_in_small || (!prefill && !fp8 && !copy_x)) return cudaSuccess;
+    return (prefill || copy_x) ? stage(slot_row, A) : stage(nullptr, T);
   }
   permute_count_kernel<<<p.nblk, kPermuteTokens, mask_bytes, st>>>(topk_idx, T, k, E, counts, lrank, status);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;

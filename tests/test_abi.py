@@ -85,7 +85,9 @@ def test_workspace_layout_is_consistent(L):
         offs = [lay.status, lay.hdr, lay.cnt, lay.mt_base, lay.row_src, lay.slot_row, lay.h, lay.y]
         assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
         assert lay.y + lay.m_rows * 2048 * 2 <= total
-        assert (lay.xa == 2 ** 64 - 1) == (path == "decode")
+        # x rows staged expert-major for the tensor-core GEMMs on both paths
+        # (tile-padded on PREFILL, one row per assignment on DECODE)
+        assert lay.xa != 2 ** 64 - 1 and lay.h - lay.xa >= lay.m_rows * 2048 * 2
 
 
 def test_e4m3_workspace_layouts(L):
@@ -106,12 +108,13 @@ def test_e4m3_workspace_layouts(L):
 
 
 def test_auto_path_choice(L):
-    """The decode-stage switch: streaming while T*k <= 2E (bf16, FP4) or
-    2*T*k <= E (e4m3), the grouped GEMMs beyond; the boundary cases included."""
+    """The decode-stage switch: the DECODE path while T*k <= 32E (bf16),
+    T*k <= 2E (FP4) or 2*T*k <= E (e4m3), the grouped GEMMs beyond; the
+    boundary cases included."""
     D, P = moe.PATH["decode"], moe.PATH["prefill"]
     assert moe.workspace_layout(shape(T=16, H=2048, I=1408, E=60, k=4)).path == D
-    assert moe.workspace_layout(shape(T=30, H=2048, I=1408, E=60, k=4)).path == D  # 120 = 2E
-    assert moe.workspace_layout(shape(T=31, H=2048, I=1408, E=60, k=4)).path == P
+    assert moe.workspace_layout(shape(T=480, H=2048, I=1408, E=60, k=4)).path == D  # 1920 = 32E
+    assert moe.workspace_layout(shape(T=481, H=2048, I=1408, E=60, k=4)).path == P
     assert moe.workspace_layout(shape(T=8192, H=2048, I=768, E=128, k=8)).path == P
     assert moe.workspace_layout(shape(T=16, H=7168, I=2048, E=256, k=8, wdtype="e4m3")).path == D  # 128 = E/2
     assert moe.workspace_layout(shape(T=17, H=7168, I=2048, E=256, k=8, wdtype="e4m3")).path == P

@@ -119,11 +119,11 @@ def test_bad_routing_index_is_reported_not_faulted():
     idx = idx.copy()
     idx[3, 1] = 4  # out of range
     idx[7, 1] = idx[7, 0]  # repeated expert
-    for path in ("prefill", "decode", "fused"):
+    for path in ("prefill", "fused", "decode"):
         out, ws = moe.forward(x.cuda(), torch.from_numpy(idx).cuda(), torch.from_numpy(w).cuda(), W["w_gate_up"],
                               W["w_down"], path=path)
         assert moe.read_device_status(ws) == -7
-    # the next good call on the same workspace clears the status
+    # the next good call on the same (DECODE) workspace clears the status
     idx2, w2, _ = O.route(L.numpy(), wl.k)
     moe.forward(x.cuda(), torch.from_numpy(idx2).cuda(), torch.from_numpy(w2).cuda(), W["w_gate_up"], W["w_down"],
                 workspace=ws, path="decode")
@@ -189,6 +189,26 @@ def test_full_size_bf16_every_token(name):
     assert_tokens_close(got, ref, TOKEN_REL_FRO, name)
 
 
+@pytest.mark.parametrize("T", [64, 128, 240])
+def test_decode_path_several_tokens_per_expert(T):
+    """The DECODE path's tensor-core GEMMs (an expert's tokens as the MMA's N)
+    at 4 to 16 tokens per expert on the decode-shaped layer, where AUTO sends
+    them: every token against the oracle, h element-wise on three experts, the
+    permutation and the combine given y bit-exact."""
+    wl = G.Workload("decode_mid", T, 2048, 1408, 60, 4)
+    shape = moe.make_shape(T, 2048, 1408, 60, 4, "bf16")
+    lay = moe.workspace_layout(shape)
+    assert lay.path == moe.PATH["decode"]
+    x, idx, w, W, out, ws = _forward(wl, 50 + T, "auto")
+    lay, perm = check_permutation(ws, shape, idx)
+    check_combine_bit_exact(ws, shape, w, out)
+    _expert_block_check(ws, lay, perm, x, idx, W, wl, [0, 30, 59])
+    ref = oracle_forward_bf16(x, idx, w, W)
+    got = out.float().cpu().numpy()
+    assert_bf16_close(got, ref, f"decode T={T}")
+    assert_tokens_close(got, ref, TOKEN_REL_FRO, f"decode T={T}")
+
+
 @pytest.mark.parametrize("path", ["prefill", "decode", "fused"])
 @pytest.mark.parametrize("name", ["tiny", "decode"])
 def test_combine_bit_exact_given_y(name, path):
@@ -232,17 +252,22 @@ def test_gated_activations(name, path, act):
     assert_bf16_close(out.float().cpu().numpy(), ref, f"{name}/{path}/{act}")
 
 
-def test_fused_path_equals_decode_path_bit_for_bit():
-    """The fused single-launch forward and the DECODE kernels compute the same
-    dot products in the same order: identical outputs, and an identical
-    permutation left in the workspace."""
+def test_fused_path_matches_decode_path():
+    """The fused single-launch forward (CUDA-core dot products) and the DECODE
+    path (tensor-core GEMMs with the tokens as N) on the same inputs: outputs
+    within the bf16 tolerance of each other and of the oracle, and the same
+    permutation left in the workspace, bit for bit."""
     wl = G.WORKLOADS["decode"]
     x, idx, w, W, out_d, ws_d = _forward(wl, 41, "decode")
     _, _, _, _, out_f, ws_f = _forward(wl, 41, "fused")
-    assert torch.equal(out_d, out_f)
+    ref = oracle_forward_bf16(x, idx, w, W)
+    assert_bf16_close(out_f.float().cpu().numpy(), ref, "fused")
+    assert_bf16_close(out_d.float().cpu().numpy(), ref, "decode")
+    assert_bf16_close(out_f.float().cpu().numpy(), out_d.float().cpu().numpy().astype(np.float64), "fused vs decode")
     shape = moe.make_shape(wl.T, wl.H, wl.I, wl.E, wl.k, "bf16", "fused")
     assert moe.workspace_layout(shape).path == moe.PATH["fused"]
     check_permutation(ws_f, shape, idx)
+    check_permutation(ws_d, moe.make_shape(wl.T, wl.H, wl.I, wl.E, wl.k, "bf16", "decode"), idx)
 
 
 def test_fused_path_bounded_wait_gives_up_cleanly():
