@@ -302,10 +302,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const size_t grow0 = static_cast<size_t>(c.e) * p.b_rows_per_expert + c.n * p.b_tile_stride + row0;
       const uint8_t* srow0 = p.w_scale + grow0 * p.kscales + half;
       const uint8_t* srow1 = p.w_scale + (grow0 + p.b_second_offset) * p.kscales + half;
+      // the scale bytes of the next stage are in flight while this one converts
+      uint32_t b0_next = __ldg(srow0), b1_next = __ldg(srow1);
       for (int kb = 0; kb < p.num_kb; ++kb) {
-        // the scale bytes are read while the codes are still in flight
-        const float sc0 = ue8m0_value(__ldg(srow0 + 2 * kb));
-        const float sc1 = ue8m0_value(__ldg(srow1 + 2 * kb));
+        const float sc0 = ue8m0_value(b0_next);
+        const float sc1 = ue8m0_value(b1_next);
+        if (kb + 1 < p.num_kb) {
+          b0_next = __ldg(srow0 + 2 * (kb + 1));
+          b1_next = __ldg(srow1 + 2 * (kb + 1));
+        }
         const bool got = mbar_wait_bounded(&rfull[stage], ph, s_abort, p.dev_status, p.timeout_ns);
         if (!__all_sync(0xffffffffu, got)) {
           ok = false;
