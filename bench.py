@@ -314,10 +314,22 @@ def stage_roofline(wl, path, stage_ms, n_touched, peaks, peak_src):
             kern, src = (("decode_e4m3_down_kernel", "decode_e4m3.cu") if fp8 else
                          ("decode_fp4_down_kernel", "decode_fp4.cu") if fp4 else
                          ("small_gemm_bf16_kernel<false>", "gemm_small.cu"))
-        ach = byts / dur_s / 1e9
-        peak = peaks["hbm_gbs"]
-        out = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
-               "kernel": kern, "stage": names[s], "algorithmic_bytes": byts}
+        # the bf16 DECODE GEMMs run on the tensor cores (bf16 MMAs, an
+        # expert's tokens as N): many tokens per expert make them
+        # tensor-bound, few make them HBM-bound; the e4m3 and e2m1 ones stream
+        # on the CUDA cores
+        flops = (4 if s == 1 else 2) * A * H * I
+        t_tensor = 0.0 if (fp8 or fp4) else flops / (peaks["bf16_tflops"] * 1e12)
+        if t_tensor > byts / (peaks["hbm_gbs"] * 1e9):
+            ach = flops / dur_s / 1e12
+            out = {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                   "frac": ach / peaks["bf16_tflops"], "peak_source": "measured bf16 burst (the MMA is bf16)",
+                   "algorithmic_flops": flops}
+        else:
+            ach = byts / dur_s / 1e9
+            peak = peaks["hbm_gbs"]
+            out = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak}
+        out.update({"kernel": kern, "stage": names[s], "algorithmic_bytes": byts})
     else:
         # the stage is bound by the tensor pipe or by HBM, whichever takes
         # longer at its measured peak: bf16 prefill shapes are tensor-bound,

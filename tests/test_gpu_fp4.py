@@ -106,20 +106,68 @@ def test_small_fp4_prefill_layer(act):
                             ExpertView(W["sw_down"], True), act=act)
     assert_bf16_close(out.float().cpu().numpy(), ref, f"fp4 prefill {act}")
     if act == "silu":
-        rows = np.nonzero(perm["row_src"] >= 0)[0]
-        h = ws_bf16(ws, lay.h, lay.m_rows, wl.I)[rows]
-        y = ws_bf16(ws, lay.y, lay.m_rows, wl.H)[rows]
-        a = perm["row_src"][rows]
-        xr = x.float().numpy()[a // wl.k]
-        e_of = idx.ravel()[a]
-        href, yref = np.zeros_like(h, dtype=np.float64), np.zeros_like(y, dtype=np.float64)
-        for e in np.unique(e_of):
-            sel = e_of == e
-            Wgu = O.dequantize_fp4(W["w_gate_up"][e].cpu().numpy(), W["sw_gate_up"][e].cpu().numpy())
-            Wd = O.dequantize_fp4(W["w_down"][e].cpu().numpy(), W["sw_down"][e].cpu().numpy())
-            href[sel], yref[sel] = O.expert_mlp(xr[sel].astype(np.float64), Wgu, Wd, "bf16")
-        assert_bf16_close(h, href, "fp4 h")
-        assert_bf16_close(y, yref, "fp4 y")
+        check_h_y(ws, lay, perm, x, idx, W, wl, "fp4 prefill")
+
+
+def check_h_y(ws, lay, perm, x, idx, W, wl, what, act="silu"):
+    """h and y of every permuted row against the oracle's expert MLP on the
+    dequantised weights."""
+    rows = np.nonzero(perm["row_src"] >= 0)[0]
+    h = ws_bf16(ws, lay.h, lay.m_rows, wl.I)[rows]
+    y = ws_bf16(ws, lay.y, lay.m_rows, wl.H)[rows]
+    a = perm["row_src"][rows]
+    xr = x.float().numpy()[a // wl.k]
+    e_of = idx.ravel()[a]
+    href, yref = np.zeros_like(h, dtype=np.float64), np.zeros_like(y, dtype=np.float64)
+    for e in np.unique(e_of):
+        sel = e_of == e
+        Wgu = O.dequantize_fp4(W["w_gate_up"][e].cpu().numpy(), W["sw_gate_up"][e].cpu().numpy())
+        Wd = O.dequantize_fp4(W["w_down"][e].cpu().numpy(), W["sw_down"][e].cpu().numpy())
+        href[sel], yref[sel] = O.expert_mlp(xr[sel].astype(np.float64), Wgu, Wd, "bf16", act=act)
+    assert_bf16_close(h, href, f"{what} h")
+    assert_bf16_close(y, yref, f"{what} y")
+
+
+@pytest.mark.parametrize("counts", [[0, 1, 127, 128, 129, 255, 256, 257, 300, 15], [16, 0, 130, 0]])
+def test_fp4_decode_path_many_tokens(counts):
+    """The DECODE path with many tokens per expert (its kernels take an
+    expert's tokens four at a time, so every tail length shows up): 0, 1,
+    127..129, 255..257 and 300 tokens; h and y of every row against the oracle."""
+    T = sum(counts)
+    wl = G.Workload("fp4many", T, 256, 384, len(counts), 1, wdtype="e2m1")
+    idx, w = G.routed_inputs_with_counts(wl, counts, seed=11)
+    x, idx_np, w_np, W, out, ws = _run(wl, 9, idx.numpy(), w.numpy(), path="decode")
+    shape = moe.make_shape(T, wl.H, wl.I, wl.E, 1, "e2m1", "decode")
+    lay, perm = check_permutation(ws, shape, idx_np)
+    check_combine_bit_exact(ws, shape, w_np, out)
+    assert_bf16_close(out.float().cpu().numpy(), oracle_fp4(x, idx_np, w_np, W), f"fp4 decode {counts}")
+    check_h_y(ws, lay, perm, x, idx_np, W, wl, f"fp4 decode {counts}")
+
+
+@pytest.mark.parametrize("path", ["decode", "prefill"])
+@pytest.mark.parametrize("which,shift,bvals", [("sw_gate_up", 100, (2, 3, 4)),
+                                               ("sw_gate_up", -18, (140, 141, 142, 143, 144, 145)),
+                                               ("sw_down", 0, (140, 141, 142, 143, 144, 145))])
+def test_fp4_scale_bytes_at_the_widening_edges(path, which, shift, bvals):
+    """Scale bytes far from those of N(0, 0.02) weights, small (2..4) and large
+    (140..145), on both paths: every weight must act as e2m1 * 2^(b-127)
+    exactly. x is scaled by 2^shift (exact in bf16) so every product and sum
+    stays a normal fp32 number; h and y of every row against the oracle."""
+    wl = G.Workload("fp4edge_scales", 40, 256, 256, 4, 2, wdtype="e2m1")
+    x, L, W = device_inputs(wl, 6)
+    x = (x.float() * 2.0 ** shift).to(torch.bfloat16)
+    rng = np.random.default_rng(abs(shift) + len(bvals))
+    W[which] = torch.from_numpy(rng.choice(np.array(bvals, dtype=np.uint8), size=tuple(W[which].shape))).to(
+        W[which].device)
+    idx, w, _ = O.route(L.numpy(), wl.k)
+    out, ws = moe.forward(x.cuda(), torch.from_numpy(idx).cuda(), torch.from_numpy(w).cuda(), W["w_gate_up"],
+                          W["w_down"], W["sw_gate_up"], W["sw_down"], path=path)
+    torch.cuda.synchronize()
+    assert moe.read_device_status(ws) == 0
+    shape = moe.make_shape(wl.T, wl.H, wl.I, wl.E, wl.k, "e2m1", path)
+    lay, perm = check_permutation(ws, shape, idx)
+    assert_bf16_close(out.float().cpu().numpy(), oracle_fp4(x, idx, w, W), f"fp4 scales {which} {bvals}")
+    check_h_y(ws, lay, perm, x, idx, W, wl, f"fp4 scales {which} {bvals}")
 
 
 @pytest.mark.parametrize("counts", [[0, 1, 127, 128, 129, 255, 256, 0], [300, 0, 0, 0, 0, 0, 0, 0]])
@@ -136,8 +184,9 @@ def test_fp4_prefill_edge_counts(counts):
 
 def test_fp4_full_size_every_token():
     """The large layer's shape with FP4 experts (T=4096, H=7168, I=2048, E=256,
-    k=8) in the launch configuration the benchmark times: every token against
-    the oracle, as a whole and token by token; permutation and combine bit-exact."""
+    k=8) in the launch configuration the benchmark times (the AUTO path), and
+    the same routing through the other path: every token against the oracle,
+    as a whole and token by token; permutation and combine bit-exact."""
     wl = G.WORKLOADS["fp4"]
     x, L, W = device_inputs(wl, G.default_seed(wl))
     layer = moe.MoELayer(W["w_gate_up"], W["w_down"], wl.k, W["sw_gate_up"], W["sw_down"])
@@ -146,14 +195,26 @@ def test_fp4_full_size_every_token():
     ws = layer._workspace(wl.T, x.cuda().device)
     assert moe.read_device_status(ws) == 0
     shape = moe.make_shape(wl.T, wl.H, wl.I, wl.E, wl.k, "e2m1")
-    assert moe.workspace_layout(shape).path == moe.PATH["prefill"]
+    auto = moe.workspace_layout(shape).path
     idx, w, _ = O.route(L.numpy(), wl.k)
     check_permutation(ws, shape, idx)
-    check_combine_bit_exact(ws, shape, device_topk_w(L, wl.k, idx), out)
+    w_dev = device_topk_w(L, wl.k, idx)
+    check_combine_bit_exact(ws, shape, w_dev, out)
     ref = oracle_fp4(x, idx, w, W, cache=False)
     got = out.float().cpu().numpy()
     assert_bf16_close(got, ref, "fp4 full")
     assert_tokens_close(got, ref, TOKEN_REL_FRO, "fp4 full")
+    other = "prefill" if auto == moe.PATH["decode"] else "decode"
+    out2, ws2 = moe.forward(x.cuda(), torch.from_numpy(idx).cuda(), torch.from_numpy(w_dev).cuda(), W["w_gate_up"],
+                            W["w_down"], W["sw_gate_up"], W["sw_down"], path=other)
+    torch.cuda.synchronize()
+    assert moe.read_device_status(ws2) == 0
+    shape2 = moe.make_shape(wl.T, wl.H, wl.I, wl.E, wl.k, "e2m1", other)
+    check_permutation(ws2, shape2, idx)
+    check_combine_bit_exact(ws2, shape2, w_dev, out2)
+    got2 = out2.float().cpu().numpy()
+    assert_bf16_close(got2, ref, f"fp4 full {other}")
+    assert_tokens_close(got2, ref, TOKEN_REL_FRO, f"fp4 full {other}")
 
 
 @pytest.mark.parametrize("T", [16, 300])
