@@ -20,9 +20,9 @@
 // routed from shared memory by one warp per token. Rows beyond E in the padded
 // tile are zero (TMA fills out-of-range rows with zeros) and never read.
 //
-// Warp roles (512 threads): warp 0 TMA producer, warp 1 TMEM allocator and
+// Warp roles (1024 threads): warp 0 TMA producer, warp 1 TMEM allocator and
 // MMA issuer, warps 2..5 epilogue (warp w reads TMEM lanes 32*(w%4)..+31);
-// then all sixteen warps route the CTA's share of the tokens.
+// then all 32 warps route the CTA's share of the tokens, one warp per token.
 #include <algorithm>
 
 #include "moe_common.cuh"
@@ -35,7 +35,7 @@ namespace {
 constexpr int kBK = 64;       // K elements per stage (128 bytes of bf16: one swizzle row)
 constexpr int kMaxStages = 8;
 constexpr size_t kRingBytes = 192 * 1024;  // shared memory for the TMA ring
-constexpr int kThreads = 512;
+constexpr int kThreads = 1024;
 constexpr int kWarps = kThreads / 32;
 constexpr int kRows = 128;    // tokens per tile (MMA M)
 constexpr int kA = kRows * kBK * 2;  // 16 KB
@@ -245,11 +245,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // Cluster size: the largest of 8, 4, 2 whose clusters (one per 128-token tile)
-// the device holds at once, that leaves every CTA at least one K block and no
-// fewer tokens per CTA than warps; else 1.
+// the device holds at once and that leaves every CTA at least one K block
+// (and at least 16 of the tile's tokens to route); else 1.
 int router_cluster_size(const void* kernel, int tiles, int num_kb, size_t smem) {
   for (int c = kMaxCluster; c > 1; c >>= 1) {
-    if (c > num_kb || kRows / c < kWarps) continue;
+    if (c > num_kb || kRows / c < 16) continue;
     const int n = max_active_clusters(kernel, c, kThreads, smem);
     if (n > 0 && tiles <= n) return c;
   }
