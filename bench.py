@@ -8,7 +8,8 @@ moe_route (router top-k) followed by moe_forward (permute, gate/up with
 SwiGLU, down, combine) of one layer. The headline workload is the large FP8
 layer (T=4096, H=7168, I=2048, E=256, k=8, e4m3 experts with UE8M0 block
 scales), the largest of the layers; the line's top-level numbers are its own.
-Every other workload (tiny, decode, prefill, skewed, fp8_decode) is measured
+Every other workload (tiny, decode, prefill, skewed, fp8_decode, fp4,
+fp4_decode) is measured
 the same way in the same process and reported under "per_config" (--only
 skips them; --workload picks another headline).
 
@@ -23,7 +24,10 @@ Each workload's entry carries: tokens/s and TFLOP/s, the stage breakdown
 (events recorded by moe_forward_timed), the roofline of the dominant kernel
 (algorithmic bytes or FLOPs per launch over its measured duration, against
 MEASURED_PEAKS.json), the end-to-end number through the public API with host
-buffers (H2D of x and logits, D2H of the output inside the timed region),
+buffers (H2D of x and logits, D2H of the output inside the timed region:
+batches pipelined through MoEPipeline, copies overlapping the previous and
+next batch's compute, where a step streams more than twice L2; else one batch
+at a time with L2 flushed between them; the other mode's figure rides along),
 the CPU oracle timed on a bounded sample (rank 0, N=1), the number of our
 kernel launches in the timed region, and the SM clocks sampled while the
 GPU was busy with it.
@@ -57,6 +61,7 @@ DEFAULT_WORKLOAD = "fp8"
 OTHER_WORKLOADS = ["tiny", "decode", "prefill", "skewed", "fp8_decode", "fp4", "fp4_decode"]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FLUSH_BYTES = 256 << 20
+L2_BYTES = 126 << 20  # B200 L2
 
 # DRAM bytes (read + write) per launch of the dominant kernel, from one ncu
 # capture each; a record counts only while its kernel's source file is
@@ -493,11 +498,12 @@ def measure(moe, wl, args, world, rank, local, peaks, peak_src):
     route_ms = sum(st_s[i].elapsed_time(st_ev[i][0]) for i in range(K)) / K
     eager_ms = sum(st_s[i].elapsed_time(st_ev[i][4]) for i in range(K)) / K
 
-    # end to end through the public API with host buffers: H2D of x and logits
-    # into the graph's inputs, the graph, D2H of the output
+    # end to end through the public API with host buffers. Serial: per step,
+    # H2D of x and logits into the graph's inputs, the graph, D2H of the
+    # output, on one stream (L2 flushed before each step, outside the events).
     xh = x.pin_memory()
     lh = logits.pin_memory()
-    oh = torch.empty((wl.T, wl.H), dtype=torch.bfloat16).pin_memory()
+    oh = [torch.empty((wl.T, wl.H), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
     e2e_s, e2e_e = new_events(K), new_events(K)
     barrier(world)
     torch.cuda.synchronize()
@@ -505,14 +511,43 @@ def measure(moe, wl, args, world, rank, local, peaks, peak_src):
         flush.zero_()
         e2e_s[i].record(stream)
         res = graph(xh, lh)
-        oh.copy_(res, non_blocking=True)
+        oh[0].copy_(res, non_blocking=True)
         e2e_e[i].record(stream)
     torch.cuda.synchronize()
     barrier(world)
-    clk = clocks.stop()
-    e2e_ms = max_over_ranks(sum(e2e_s[i].elapsed_time(e2e_e[i]) for i in range(K)), world)
-    if not torch.equal(graph.out, out):
+    e2e_serial_ms = max_over_ranks(sum(e2e_s[i].elapsed_time(e2e_e[i]) for i in range(K)), world)
+    if not torch.equal(graph.out, out) or not torch.equal(oh[0], out.cpu()):
         raise RuntimeError("graph replay and eager forward disagree")
+    # Pipelined (MoEPipeline): batch i's copy-in and batch i-1's copy-out
+    # overlap batch i's graph; one device-timed span from the first copy-in to
+    # the last copy-out. Larger layers stream more than L2 every step, so the
+    # span needs no flush; where the touched weights fit twice in L2 the flush
+    # has to run on the compute stream before every batch, inside the span,
+    # and the serial figure (flush outside the events) is the e2e value.
+    weight_bytes = n_touched * 3 * wl.H * wl.I * {"e4m3": 1, "e2m1": 0.5}.get(wl.wdtype, 2)
+    flush_inside = weight_bytes < 2 * L2_BYTES
+    pipe = moe.MoEPipeline(layer, wl.T, dev)
+    hook = flush.zero_ if flush_inside else None
+    for i in range(max(args.warmup, 2)):
+        pipe.submit(xh, lh, oh[i % 2], before_compute=hook)
+    pipe.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    ev0.record(pipe.copy_in)
+    for i in range(K):
+        pipe.submit(xh, lh, oh[i % 2], before_compute=hook)
+    pipe.compute.wait_stream(pipe.copy_in)
+    pipe.copy_out.wait_stream(pipe.compute)
+    ev1.record(pipe.copy_out)
+    pipe.synchronize()
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    e2e_ms = max_over_ranks(ev0.elapsed_time(ev1), world)
+    if not (torch.equal(oh[0], out.cpu()) and torch.equal(oh[1], out.cpu())):
+        raise RuntimeError("pipelined steps and eager forward disagree")
+    del pipe
 
     router_line = None
     if args.router and wl.E <= 256:
@@ -540,8 +575,17 @@ def measure(moe, wl, args, world, rank, local, peaks, peak_src):
                       "combine": stage_ms[4], "eager_step": eager_ms},
         "touched_experts": n_touched,
         "roofline": stage_roofline(wl, path, {1: stage_ms[2], 2: stage_ms[3]}, n_touched, peaks, peak_src),
-        "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s",
-                "h2d_bytes_per_step": x.numel() * 2 + logits.numel() * 4, "d2h_bytes_per_step": wl.T * wl.H * 2},
+        "e2e": ({"value": tokens / (e2e_serial_ms / 1e3), "unit": "tokens/s",
+                 "h2d_bytes_per_step": x.numel() * 2 + logits.numel() * 4, "d2h_bytes_per_step": wl.T * wl.H * 2,
+                 "mode": "serial: copy-in, graph, copy-out on one stream per step, L2 flushed between steps",
+                 "pipelined_value": tokens / (e2e_ms / 1e3),
+                 "pipelined_l2": "flushed before every batch inside the span"}
+                if flush_inside else
+                {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s",
+                 "h2d_bytes_per_step": x.numel() * 2 + logits.numel() * 4, "d2h_bytes_per_step": wl.T * wl.H * 2,
+                 "mode": "MoEPipeline: copy-in, graph and copy-out on three streams, two batches in flight",
+                 "l2": f"not flushed: each step streams {weight_bytes / 1e9:.2f} GB of weights, more than L2",
+                 "serial_value": tokens / (e2e_serial_ms / 1e3)}),
         "gpu_launches": per_step_launches * K,
         "clocks": clk,
     }

@@ -377,6 +377,73 @@ class MoEGraph:
         return self.replay()
 
 
-__all__ = ["lib", "route", "forward", "forward_noalloc", "noalloc_device_status", "MoEGraph", "workspace_size", "workspace_layout", "alloc_workspace",
+class MoEPipeline:
+    """Layer steps from host memory to host memory for a stream of batches,
+    with the copies overlapped with the compute: batch i's x and logits are
+    copied in on one stream while batch i-1 runs, and batch i-1's output is
+    copied out on another while batch i runs. ``depth`` MoEGraph instances
+    (static device buffers and a captured graph each) take the batches in
+    turn; their graphs run in submission order on one compute stream, so they
+    share the layer's workspace. Events keep a buffer set from being refilled
+    before its graph has read it and its output from being overwritten before
+    it was copied out. Host tensors must be pinned for the copies to overlap;
+    a caller reads ``out_host`` of a batch after ``done(i)`` or ``synchronize()``."""
+
+    def __init__(self, layer: "MoELayer", T: int, device=None, depth: int = 2):
+        if depth < 2:
+            raise ValueError("depth must be at least 2 for the copies to overlap the compute")
+        device = torch.device(device or "cuda")
+        self.device = device
+        self.depth = depth
+        self.graphs = [MoEGraph(layer, T, device) for _ in range(depth)]
+        self.copy_in = torch.cuda.Stream(device=device)
+        self.compute = torch.cuda.Stream(device=device)
+        self.copy_out = torch.cuda.Stream(device=device)
+        self.inputs_ready = [torch.cuda.Event() for _ in range(depth)]
+        self.computed = [torch.cuda.Event() for _ in range(depth)]
+        self.output_read = [torch.cuda.Event() for _ in range(depth)]
+        self.n = 0
+
+    def submit(self, x_host: torch.Tensor, logits_host: torch.Tensor, out_host: torch.Tensor, before_compute=None):
+        """Queue one batch; returns its sequence number. ``before_compute``, if
+        given, is called with the compute stream current just before the
+        batch's graph (for work that must run in the compute order)."""
+        s = self.n % self.depth
+        g = self.graphs[s]
+        reuse = self.n >= self.depth
+        with torch.cuda.stream(self.copy_in):
+            if reuse:
+                self.copy_in.wait_event(self.computed[s])  # the slot's previous graph has read its inputs
+            g.x.copy_(x_host, non_blocking=True)
+            g.logits.copy_(logits_host, non_blocking=True)
+            self.inputs_ready[s].record(self.copy_in)
+        with torch.cuda.stream(self.compute):
+            self.compute.wait_event(self.inputs_ready[s])
+            if reuse:
+                self.compute.wait_event(self.output_read[s])  # the slot's previous output was copied out
+            if before_compute is not None:
+                before_compute()
+            g.graph.replay()
+            self.computed[s].record(self.compute)
+        with torch.cuda.stream(self.copy_out):
+            self.copy_out.wait_event(self.computed[s])
+            out_host.copy_(g.out, non_blocking=True)
+            self.output_read[s].record(self.copy_out)
+        self.n += 1
+        return self.n - 1
+
+    def done(self, i: int) -> bool:
+        """True once batch i's output has been copied out (only the last
+        ``depth`` batches can be asked)."""
+        if not (self.n - self.depth <= i < self.n):
+            raise ValueError("only the last depth batches can be queried")
+        return self.output_read[i % self.depth].query()
+
+    def synchronize(self):
+        for st in (self.copy_in, self.compute, self.copy_out):
+            st.synchronize()
+
+
+__all__ = ["lib", "route", "forward", "forward_noalloc", "noalloc_device_status", "MoEGraph", "MoEPipeline", "workspace_size", "workspace_layout", "alloc_workspace",
            "read_device_status", "set_test_hooks", "router", "make_shape", "MoELayer", "MoeError", "MoeShape", "EXPORTS", "STATUS",
            "status_string", "PATH", "WDTYPE", "ACT"]
