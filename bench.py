@@ -73,6 +73,16 @@ NCU_TRAFFIC = {
                                                          "scaled": None},
     ("fp8", "grouped_gemm_e4m3_kernel<true>"): {"bytes": 8316361440, "src": "dc4eb5e6a4256cd9",
                                                 "scaled": "T=1024, E=64 capture x4 (rows and experts)"},
+    ("skewed", "grouped_gemm_bf16_kernel<256,true>"): {"bytes": 2192461184, "src": "d64f0e084cc41143",
+                                                        "scaled": None},
+    ("fp8_decode", "decode_e4m3_gate_up_kernel"): {
+        "bytes": 2907074829, "src": "a9ccd1d763968d66",
+        "scaled": "T=16, E=64 capture (59 experts touched) x 1.593, the ratio of algorithmic bytes (94 touched)"},
+    ("fp4", "grouped_gemm_fp4_kernel<1,0>"): {"bytes": 6701524992, "src": "1c31b7fc99a0883e",
+                                             "scaled": "T=1024, E=64 capture x4 (rows and experts)"},
+    ("fp4_decode", "decode_fp4_gate_up_kernel"): {
+        "bytes": 1769561034, "src": "9b2030e9dee1e2d9",
+        "scaled": "T=16, E=64 capture (59 experts touched) x 1.627, the ratio of algorithmic bytes (96 touched)"},
 }
 
 
