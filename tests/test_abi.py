@@ -284,3 +284,11 @@ def test_binding_requires_one_device():
     with pytest.raises(ValueError, match="on a CUDA device"):
         moe._same_device(torch.device("cpu"))
     moe._same_device(dev, out=None)  # absent tensors are fine
+
+
+def test_pipeline_needs_two_batches_in_flight():
+    """MoEPipeline overlaps the copies of neighbouring batches with the
+    compute only with at least two buffer sets; fewer is refused before any
+    device work."""
+    with pytest.raises(ValueError):
+        moe.MoEPipeline(None, 16, depth=1)
