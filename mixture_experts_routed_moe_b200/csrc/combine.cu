@@ -21,6 +21,8 @@ __global__ void __launch_bounds__(kBlock) combine_kernel(const __nv_bfloat16* __
                                                          const int* __restrict__ slot_row,
                                                          const float* __restrict__ topk_w,
                                                          __nv_bfloat16* __restrict__ out, int H, int k) {
+  pdl_wait();  // the previous kernel on the stream has completed; its writes are visible
+  pdl_trigger();
   extern __shared__ int s_slot[];  // [k] rows, then [k] weights
   float* s_w = reinterpret_cast<float*>(s_slot + k);
   const int t = blockIdx.x;
@@ -68,10 +70,9 @@ __global__ void __launch_bounds__(kBlock) combine_kernel(const __nv_bfloat16* __
 cudaError_t launch_combine(const moe_shape* s, const Plan& p, const float* topk_w, void* out, uint8_t* ws,
                            cudaStream_t st) {
   const size_t smem = static_cast<size_t>(s->k) * (sizeof(int) + sizeof(float));  // k <= 1024: at most 8 KB
-  combine_kernel<<<s->T, kBlock, smem, st>>>(reinterpret_cast<const __nv_bfloat16*>(ws + p.y),
-                                          reinterpret_cast<const int*>(ws + p.slot_row), topk_w,
-                                          static_cast<__nv_bfloat16*>(out), s->H, s->k);
-  return cudaGetLastError();
+  return launch_pdl(combine_kernel, dim3(s->T), dim3(kBlock), smem, st,
+                    reinterpret_cast<const __nv_bfloat16*>(ws + p.y), reinterpret_cast<const int*>(ws + p.slot_row),
+                    topk_w, static_cast<__nv_bfloat16*>(out), s->H, s->k);
 }
 
 }  // namespace moe

@@ -115,6 +115,8 @@ __global__ void __launch_bounds__(kBlock, 2) decode_e4m3_gate_up_kernel(
     const uint8_t* __restrict__ sgu, const int* __restrict__ cnt, const int* __restrict__ row_off,
     const int* __restrict__ row_src, const int* __restrict__ touched, const int* __restrict__ hdr,
     float* __restrict__ hf, int H, int I, int k, int act) {
+  pdl_wait();  // the previous kernel on the stream has completed; its writes are visible
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int gwarp = blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
   const int nwarps = gridDim.x * kWarpsPerBlock;
@@ -165,6 +167,8 @@ __global__ void __launch_bounds__(kBlock, 2) decode_e4m3_gate_up_kernel(
 __global__ void __launch_bounds__(kBlock) decode_e4m3_quant_h_kernel(const float* __restrict__ hf,
                                                                       uint8_t* __restrict__ hq,
                                                                       float* __restrict__ hs, long long rows, int I) {
+  pdl_wait();  // the previous kernel on the stream has completed; its writes are visible
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const long long gwarp = static_cast<long long>(blockIdx.x) * kWarpsPerBlock + (threadIdx.x >> 5);
   const long long nwarps = static_cast<long long>(gridDim.x) * kWarpsPerBlock;
@@ -214,6 +218,8 @@ __global__ void __launch_bounds__(kBlock, 2) decode_e4m3_down_kernel(
     const uint8_t* __restrict__ hq, const float* __restrict__ hs, const uint8_t* __restrict__ wd,
     const uint8_t* __restrict__ sd, const int* __restrict__ cnt, const int* __restrict__ row_off,
     const int* __restrict__ touched, const int* __restrict__ hdr, __nv_bfloat16* __restrict__ y, int H, int I) {
+  pdl_wait();  // the previous kernel on the stream has completed; its writes are visible
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int gwarp = blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
   const int nwarps = gridDim.x * kWarpsPerBlock;
@@ -290,24 +296,22 @@ cudaError_t launch_decode_e4m3(const moe_shape* s, const Plan& p, const void* w_
   if (which == 0) {
     err = one_wave(decode_e4m3_gate_up_kernel, &per_sm[0], num_sms, &grid);
     if (err != cudaSuccess) return err;
-    decode_e4m3_gate_up_kernel<<<grid, kBlock, 0, st>>>(xq, xs, static_cast<const uint8_t*>(w_gate_up),
-                                                        sw_gate_up, cnt, row_off, row_src, touched, hdr, hf, s->H,
-                                                        s->I, s->k, s->act);
-    err = cudaGetLastError();
+    err = launch_pdl(decode_e4m3_gate_up_kernel, dim3(grid), dim3(kBlock), 0, st, xq, xs,
+                     static_cast<const uint8_t*>(w_gate_up), sw_gate_up, cnt, row_off, row_src, touched, hdr, hf, s->H,
+                     s->I, s->k, s->act);
     if (err != cudaSuccess) return err;
     err = one_wave(decode_e4m3_quant_h_kernel, &per_sm[1], num_sms, &grid);
     if (err != cudaSuccess) return err;
     const long long groups = p.m_rows * (s->I / 128);
     const long long need = (groups + kWarpsPerBlock - 1) / kWarpsPerBlock;
     grid = static_cast<int>(need < grid ? (need < 1 ? 1 : need) : grid);
-    decode_e4m3_quant_h_kernel<<<grid, kBlock, 0, st>>>(hf, hq, hs, p.m_rows, s->I);
+    return launch_pdl(decode_e4m3_quant_h_kernel, dim3(grid), dim3(kBlock), 0, st, hf, hq, hs, p.m_rows, s->I);
   } else {
     err = one_wave(decode_e4m3_down_kernel, &per_sm[2], num_sms, &grid);
     if (err != cudaSuccess) return err;
-    decode_e4m3_down_kernel<<<grid, kBlock, 0, st>>>(hq, hs, static_cast<const uint8_t*>(w_down), sw_down, cnt,
-                                                     row_off, touched, hdr, y, s->H, s->I);
+    return launch_pdl(decode_e4m3_down_kernel, dim3(grid), dim3(kBlock), 0, st, hq, hs,
+                      static_cast<const uint8_t*>(w_down), sw_down, cnt, row_off, touched, hdr, y, s->H, s->I);
   }
-  return cudaGetLastError();
 }
 
 }  // namespace moe

@@ -145,6 +145,8 @@ __global__ void __launch_bounds__(kBlock, 2) decode_fp4_gate_up_kernel(
     const int* __restrict__ cnt, const int* __restrict__ row_off, const int* __restrict__ row_src,
     const int* __restrict__ touched, const int* __restrict__ hdr, __nv_bfloat16* __restrict__ h, int H, int I, int k,
     int act) {
+  pdl_wait();  // the previous kernel on the stream has completed; its writes are visible
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int gwarp = blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
   const int nwarps = gridDim.x * kWarpsPerBlock;
@@ -181,6 +183,8 @@ __global__ void __launch_bounds__(kBlock, 2) decode_fp4_down_kernel(
     const __nv_bfloat16* __restrict__ h, const uint8_t* __restrict__ wd, const uint8_t* __restrict__ sd,
     const int* __restrict__ cnt, const int* __restrict__ row_off, const int* __restrict__ touched,
     const int* __restrict__ hdr, __nv_bfloat16* __restrict__ y, int H, int I) {
+  pdl_wait();  // the previous kernel on the stream has completed; its writes are visible
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int gwarp = blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
   const int nwarps = gridDim.x * kWarpsPerBlock;
@@ -235,14 +239,12 @@ cudaError_t launch_decode_fp4(const moe_shape* s, const Plan& p, const void* x, 
   }
   const int grid = num_sms * per_sm[which];
   if (which == 0) {
-    decode_fp4_gate_up_kernel<<<grid, kBlock, 0, st>>>(static_cast<const __nv_bfloat16*>(x),
-                                                       static_cast<const uint8_t*>(w_gate_up), sw_gate_up, cnt,
-                                                       row_off, row_src, touched, hdr, h, s->H, s->I, s->k, s->act);
-  } else {
-    decode_fp4_down_kernel<<<grid, kBlock, 0, st>>>(h, static_cast<const uint8_t*>(w_down), sw_down, cnt, row_off,
-                                                    touched, hdr, y, s->H, s->I);
+    return launch_pdl(decode_fp4_gate_up_kernel, dim3(grid), dim3(kBlock), 0, st, static_cast<const __nv_bfloat16*>(x),
+                      static_cast<const uint8_t*>(w_gate_up), sw_gate_up, cnt, row_off, row_src, touched, hdr, h, s->H,
+                      s->I, s->k, s->act);
   }
-  return cudaGetLastError();
+  return launch_pdl(decode_fp4_down_kernel, dim3(grid), dim3(kBlock), 0, st, h, static_cast<const uint8_t*>(w_down),
+                    sw_down, cnt, row_off, touched, hdr, y, s->H, s->I);
 }
 
 }  // namespace moe

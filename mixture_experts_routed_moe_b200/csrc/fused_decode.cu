@@ -133,6 +133,8 @@ __device__ __forceinline__ int block_scan(int v, int* s_warp) {
 }
 
 __global__ void __launch_bounds__(kBlock) fused_decode_kernel(const FusedParams p) {
+  pdl_wait();  // the previous kernel on the stream has completed; its writes are visible
+  pdl_trigger();
   extern __shared__ int smem_i[];
   const int E = p.E, T = p.T, k = p.k, H = p.H, I = p.I;
   const int A = T * k;
@@ -370,8 +372,7 @@ cudaError_t launch_fused_decode(const moe_shape* s, const Plan& p, const void* x
   if (err != cudaSuccess) return err;
   err = cudaMemsetAsync(fp.sync, 0, static_cast<size_t>(3 + 2 * s->E) * sizeof(int), st);
   if (err != cudaSuccess) return err;
-  fused_decode_kernel<<<num_sms * std::max(1, per_sm), kBlock, smem, st>>>(fp);
-  return cudaGetLastError();
+  return launch_pdl(fused_decode_kernel, dim3(num_sms * std::max(1, per_sm)), dim3(kBlock), smem, st, fp);
 }
 
 }  // namespace moe

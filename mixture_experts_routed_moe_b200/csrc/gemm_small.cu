@@ -92,6 +92,8 @@ template <bool kGateUp, int kAct>
 __global__ void __launch_bounds__(kThreads, 1)
     small_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                            const SmallParams p) {
+  pdl_wait();  // the previous kernel on the stream has completed; its writes are visible
+  pdl_trigger();
   using C = SmallCfg<kGateUp>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -272,8 +274,7 @@ cudaError_t launch_small_t(const CUtensorMap& tmW, const CUtensorMap& tmX, const
   static unsigned long long done = 0;
   cudaError_t err = ensure_max_smem(reinterpret_cast<const void*>(small_gemm_bf16_kernel<kGateUp, kAct>), &done);
   if (err != cudaSuccess) return err;
-  small_gemm_bf16_kernel<kGateUp, kAct><<<grid, kThreads, C::kSmem, st>>>(tmW, tmX, sp);
-  return cudaGetLastError();
+  return launch_pdl(small_gemm_bf16_kernel<kGateUp, kAct>, dim3(grid), dim3(kThreads), C::kSmem, st, tmW, tmX, sp);
 }
 
 }  // namespace

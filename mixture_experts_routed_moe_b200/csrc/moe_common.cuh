@@ -22,6 +22,17 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// Programmatic dependent launch. A kernel launched with programmatic stream
+// serialization (launch_pdl) may become resident while the previous kernel
+// on the stream is still running; pdl_wait() returns once that kernel has
+// completed and its memory operations are visible, so it comes before any
+// global memory access of the kernel. pdl_trigger() lets the next kernel of
+// the stream be launched once every block of this one has started (it still
+// waits for this one to complete before touching memory). Both are no-ops
+// for an ordinary launch.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

@@ -123,4 +123,24 @@ cudaError_t ensure_max_smem(const void* kernel, unsigned long long* done);
 // cluster grid larger than this leaves clusters waiting for a second wave.
 int max_active_clusters(const void* kernel, int cluster, int threads, size_t smem);
 
+// Launches `kernel` with programmatic stream serialization: it may become
+// resident while the previous kernel on the stream finishes, and waits for it
+// with pdl_wait() before touching memory (every kernel launched this way
+// does so first). Saves the launch gap between short kernels.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+}
+
 }  // namespace moe

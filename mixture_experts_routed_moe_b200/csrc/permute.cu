@@ -54,6 +54,8 @@ __global__ void __launch_bounds__(kPermuteTokens) permute_count_kernel(const int
                                                                        int E, int* __restrict__ block_counts,
                                                                        int* __restrict__ local_rank,
                                                                        int* dev_status) {
+  pdl_wait();  // the previous kernel on the stream has completed; its writes are visible
+  pdl_trigger();
   extern __shared__ uint32_t s_mask[];  // [kWarps][E]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int i = threadIdx.x; i < kWarps * E; i += kPermuteTokens) s_mask[i] = 0;
@@ -153,6 +155,8 @@ __device__ __forceinline__ void scan_experts(int* __restrict__ counts, int nblk,
 __global__ void __launch_bounds__(1024) permute_scan_kernel(int* counts, int nblk, int E, int bm, int* cnt,
                                                             int* mt_base, int* pt_base, int* touched, int* hdr,
                                                             int* row_src) {
+  pdl_wait();  // the previous kernel on the stream has completed; its writes are visible
+  pdl_trigger();
   __shared__ int s_warp[32];
   scan_experts(counts, nblk, E, bm, cnt, mt_base, pt_base, touched, hdr, row_src, s_warp);
 }
@@ -222,6 +226,8 @@ __global__ void __launch_bounds__(256) stage_rows_kernel(const __nv_bfloat16* __
                                                          const int* __restrict__ slot_row, long long n_src, int k,
                                                          int H, __nv_bfloat16* __restrict__ xa,
                                                          uint8_t* __restrict__ xq, float* __restrict__ xs) {
+  pdl_wait();  // the previous kernel on the stream has completed; its writes are visible
+  pdl_trigger();
   const int G = H / 128;
   const long long total = n_src * G;
   const int l16 = threadIdx.x & 15;
@@ -259,6 +265,8 @@ __global__ void __launch_bounds__(256) permute_scatter_kernel(const int* __restr
                                                               const __nv_bfloat16* __restrict__ x,
                                                               __nv_bfloat16* __restrict__ xa, uint8_t* __restrict__ xq,
                                                               float* __restrict__ xs, int H) {
+  pdl_wait();  // the previous kernel on the stream has completed; its writes are visible
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const long long t = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   if (t >= T) return;
@@ -327,6 +335,8 @@ __global__ void __launch_bounds__(1024) permute_small_kernel(const int* __restri
                                                              const __nv_bfloat16* __restrict__ x,
                                                              __nv_bfloat16* __restrict__ xa, uint8_t* __restrict__ xq,
                                                              float* __restrict__ xs, int H) {
+  pdl_wait();  // the previous kernel on the stream has completed; its writes are visible
+  pdl_trigger();
   extern __shared__ uint32_t s_mask[];  // [kWarps][E]
   __shared__ int s_warp[32];
   __shared__ int s_base[1024];  // per-expert block base is always 0 here; holds mt_base*bm
@@ -427,30 +437,29 @@ cudaError_t launch_permute(const moe_shape* s, const Plan& p, const int* topk_id
     const long long want = (tasks + 15) / 16;  // blocks of 16 half-warps
     const long long cap = static_cast<long long>(device_sm_count()) * 8;
     const unsigned grid = static_cast<unsigned>(std::max<long long>(1, std::min(want, cap)));
-    stage_rows_kernel<<<grid, 256, 0, st>>>(xb, slots, n_src, k, H, xa, xq, xs);
-    return cudaGetLastError();
+    return launch_pdl(stage_rows_kernel, dim3(grid), dim3(256), 0, st, xb, slots, n_src, k, H, xa, xq, xs);
   };
 
   cudaError_t err = cudaMemsetAsync(status, 0, kStatusWordsZeroed * sizeof(int), st);
   if (err != cudaSuccess) return err;
   if (T <= kSmallPermuteT) {
-    permute_small_kernel<<<1, 1024, mask_bytes, st>>>(topk_idx, T, k, E, p.bm, cnt, mt_base, pt_base, touched, hdr,
-                                                      row_src, slot_row, lrank, status, xb,
-                                                      stage_in_small ? xa : nullptr,
-                                                      stage_in_small ? xq : nullptr,
-                                                      stage_in_small ? xs : nullptr, H);
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    err = launch_pdl(permute_small_kernel, dim3(1), dim3(1024), mask_bytes, st, topk_idx, T, k, E, p.bm, cnt, mt_base,
+                     pt_base, touched, hdr, row_src, slot_row, lrank, status, xb, stage_in_small ? xa : nullptr,
+                     stage_in_small ? xq : nullptr, stage_in_small ? xs : nullptr, H);
+    if (err != cudaSuccess) return err;
     if (stage_in_small || (!prefill && !fp8 && !copy_x)) return cudaSuccess;
     return (prefill || copy_x) ? stage(slot_row, A) : stage(nullptr, T);
   }
-  permute_count_kernel<<<p.nblk, kPermuteTokens, mask_bytes, st>>>(topk_idx, T, k, E, counts, lrank, status);
-  if ((err = cudaGetLastError()) != cudaSuccess) return err;
-  permute_scan_kernel<<<1, 1024, 0, st>>>(counts, p.nblk, E, p.bm, cnt, mt_base, pt_base, touched, hdr, row_src);
-  if ((err = cudaGetLastError()) != cudaSuccess) return err;
-  permute_scatter_kernel<<<static_cast<unsigned>((T + 7) / 8), 256, 0, st>>>(
-      topk_idx, T, k, E, p.bm, counts, lrank, mt_base, row_src, slot_row, xb, xa, prefill ? xq : nullptr,
-      prefill ? xs : nullptr, H);
-  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  err = launch_pdl(permute_count_kernel, dim3(p.nblk), dim3(kPermuteTokens), mask_bytes, st, topk_idx, T, k, E, counts,
+                   lrank, status);
+  if (err != cudaSuccess) return err;
+  err = launch_pdl(permute_scan_kernel, dim3(1), dim3(1024), 0, st, counts, p.nblk, E, p.bm, cnt, mt_base, pt_base,
+                   touched, hdr, row_src);
+  if (err != cudaSuccess) return err;
+  err = launch_pdl(permute_scatter_kernel, dim3(static_cast<unsigned>((T + 7) / 8)), dim3(256), 0, st, topk_idx, T, k,
+                   E, p.bm, counts, lrank, mt_base, row_src, slot_row, xb, xa, prefill ? xq : nullptr,
+                   prefill ? xs : nullptr, H);
+  if (err != cudaSuccess) return err;
   return (!prefill && fp8) ? stage(nullptr, T) : cudaSuccess;
 }
 

@@ -18,6 +18,8 @@ template <int kPerLane>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32) route_kernel(const float* __restrict__ logits, int T, int E,
                                                                     int k, int* __restrict__ topk_idx,
                                                                     float* __restrict__ topk_w) {
+  pdl_wait();  // the previous kernel on the stream has completed; its writes are visible
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * kWarpsPerBlock + warp;
   if (t >= T) return;
@@ -28,8 +30,8 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) route_kernel(const float*
 template <int kPerLane>
 cudaError_t launch_route_t(const float* logits, int T, int E, int k, int* idx, float* w, cudaStream_t st) {
   const int blocks = (T + kWarpsPerBlock - 1) / kWarpsPerBlock;
-  route_kernel<kPerLane><<<blocks, kWarpsPerBlock * 32, 0, st>>>(logits, T, E, k, idx, w);
-  return cudaGetLastError();
+  return launch_pdl(route_kernel<kPerLane>, dim3(blocks), dim3(kWarpsPerBlock * 32), 0, st, logits, T, E, k, idx,
+                    w);
 }
 
 }  // namespace
